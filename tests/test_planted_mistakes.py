@@ -1,0 +1,78 @@
+"""Plant plausible slips in a copy of the oracle and check the pins catch each.
+
+The copy is built from the oracle's source text with one substitution and run
+on the CPU only; the real oracle is untouched.
+"""
+import importlib.util
+import inspect
+import sys
+import types
+
+import pytest
+
+import tests.test_oracle_pins as pins
+from oracle import mla_oracle
+
+MUTATIONS = {
+    # transposed / wrong head slice in the up-projection (eq 10)
+    "uk_transposed": ("k_c = c_kv @ W[\"w_uk\"].astype(F64).T", "k_c = c_kv @ W[\"w_uv\"].astype(F64).T"),
+    # dropped d_h^R from the softmax scale
+    "scale_drops_rope_dim": ("math.sqrt(D.d_h + D.d_hr)", "math.sqrt(D.d_h)"),
+    # wrong sign in one RoPE component
+    "rope_sign": ("out[..., 1::2] = even * s + odd * c", "out[..., 1::2] = even * s - odd * c"),
+    # RoPE position not applied to the key
+    "rope_key_unrotated": ("k_r = rope_rotate(W[\"w_kr\"].astype(F64) @ h, pos, dims_theta(D))",
+                           "k_r = W[\"w_kr\"].astype(F64) @ h"),
+    # query RoPE taken at a shifted position
+    "rope_query_pos": ("q_r = rope_rotate(q_r_pre, pos, dims_theta(D))",
+                       "q_r = rope_rotate(q_r_pre, pos + 1, dims_theta(D))"),
+    # current token left out of its own attention (eq 7 sums j <= t)
+    "causal_off_by_one": ("rows[:pos + 1])", "rows[:pos])"),
+    # absorbed query with the wrong contraction index
+    "absorb_wrong_axis": ("np.einsum(\"ihc,ih->ic\", w_uk, q_c)",
+                          "np.einsum(\"ihc,ih->ic\", w_uk, q_c[:, ::-1])"),
+    # softmax normaliser dropped
+    "softmax_unnormalised": ("return e / s, float(m + math.log(s))", "return e, float(m + math.log(s))"),
+    # log-sum-exp missing the max
+    "lse_missing_max": ("float(m + math.log(s))", "float(math.log(s))"),
+    # YaRN blend with the wrong end points
+    "yarn_blend_swapped": ("out[i] = (1.0 - g) * theta[i] / yarn_scale + g * theta[i]",
+                           "out[i] = g * theta[i] / yarn_scale + (1.0 - g) * theta[i]"),
+    # W^O applied before W^UV's head split is undone
+    "out_proj_heads": ("o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64))",
+                       "o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64)[::-1])"),
+}
+
+
+def _mutated(name):
+    src = inspect.getsource(mla_oracle)
+    old, new = MUTATIONS[name]
+    assert src.count(old) >= 1, f"mutation {name} does not match the oracle source"
+    mod = types.ModuleType(f"mla_oracle_mut_{name}")
+    exec(compile(src.replace(old, new), mod.__name__, "exec"), mod.__dict__)
+    return mod
+
+
+def _pin_tests():
+    out = []
+    for n, f in inspect.getmembers(pins, inspect.isfunction):
+        if n.startswith("test_"):
+            params = getattr(f, "pytestmark", [])
+            argsets = [()]
+            for m in params:
+                if m.name == "parametrize":
+                    argsets = [(v,) for v in m.args[1]]
+            out.extend((n, f, a) for a in argsets)
+    return out
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    monkeypatch.setattr(pins, "O", _mutated(name))
+    caught = []
+    for n, f, args in _pin_tests():
+        try:
+            f(*args)
+        except (AssertionError, ValueError, IndexError, FloatingPointError):
+            caught.append(n)
+    assert caught, f"no pin caught mutation {name}"
