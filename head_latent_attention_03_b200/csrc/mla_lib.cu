@@ -1,0 +1,223 @@
+// mla_lib.cu — the C ABI of include/mla.h (one translation unit).
+//
+// Host side of every entry point: argument validation, workspace carving,
+// TMA descriptor creation and kernel launches on the caller's stream.  The
+// kernels themselves live in the included .cuh files.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "rope.cuh"
+#include "simt_f32.cuh"
+#include "tc_kernels.cuh"
+
+using namespace mla;
+
+namespace {
+
+constexpr int kVersionMajor = 0, kVersionMinor = 1;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+mla_status_t check_launch() {
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+bool desc_valid(const mla_layer_desc* D) {
+  if (!D) return false;
+  if (D->d <= 0 || D->n_h <= 0 || D->d_h <= 0 || D->d_c <= 0 || D->d_cq < 0 || D->d_hr < 0) return false;
+  if (D->d_hr % 2 != 0 || D->block_size <= 0) return false;
+  if (!(D->rope_base > 0.0) || !(D->yarn_scale >= 1.0) || !(D->attn_logit_factor > 0.0)) return false;
+  if (D->yarn_scale > 1.0 && (D->yarn_orig_ctx <= 0 || !(D->yarn_beta > D->yarn_alpha))) return false;
+  return D->dtype == MLA_F32 || D->dtype == MLA_BF16;
+}
+
+// Shapes the tcgen05 kernels are written for.
+bool bf16_supported(const mla_layer_desc* D) {
+  return D->block_size == 64 && D->d_c == 512 && D->d_hr == 64 && D->d_h % 64 == 0 && D->d % 64 == 0 &&
+         D->d_cq % 64 == 0 && (D->n_h == 16 || D->n_h == 32 || D->n_h == 64 || D->n_h == 128);
+}
+
+RopeParams rope_params(const mla_layer_desc* D) {
+  RopeParams r;
+  r.base = D->rope_base;
+  r.yarn_scale = D->yarn_scale;
+  r.yarn_alpha = D->yarn_alpha;
+  r.yarn_beta = D->yarn_beta;
+  r.yarn_orig_ctx = D->yarn_orig_ctx;
+  return r;
+}
+
+double softmax_scale(const mla_layer_desc* D) { return D->attn_logit_factor / sqrt((double)(D->d_h + D->d_hr)); }
+
+F32Layer f32_layer(const mla_layer_desc* D) {
+  F32Layer L;
+  L.d = D->d;
+  L.n_h = D->n_h;
+  L.d_h = D->d_h;
+  L.d_c = D->d_c;
+  L.d_cq = D->d_cq;
+  L.d_hr = D->d_hr;
+  L.block_size = D->block_size;
+  L.rope = rope_params(D);
+  L.scale_log2 = (float)(softmax_scale(D) * 1.4426950408889634);
+  return L;
+}
+
+bool cache_valid(const mla_paged_cache* c) {
+  return c && c->pool && c->block_table && c->num_blocks > 0 && c->max_blocks > 0;
+}
+
+size_t f32_attn_ws(const mla_layer_desc* D, int rows, int max_len) {
+  return (size_t)rows * D->n_h * (size_t)max_len * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_version(void) { return (kVersionMajor << 16) | kVersionMinor; }
+
+const char* mla_status_string(mla_status_t s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MLA_ERR_CAPACITY: return "capacity exceeded (workspace or page id)";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t mla_workspace_size(const mla_layer_desc* D, int T, int B, int max_kv_len) {
+  if (!desc_valid(D) || T < 0 || B < 0 || max_kv_len < 0) return 0;
+  if (D->dtype == MLA_F32) {
+    const int cap = (max_kv_len + D->block_size - 1) / D->block_size * D->block_size;
+    return f32_attn_ws(D, B, cap) + 256;
+  }
+  return tc_workspace_size(D, T, B, max_kv_len);
+}
+
+mla_status_t mla_compress_append(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* seq_idx,
+                                 const int32_t* pos, int T, mla_paged_cache* cache, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!desc_valid(D) || !w || !w->w_dkv || !w->w_kr || !h || !seq_idx || !pos || T < 0 || !cache_valid(cache))
+    return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (D->dtype == MLA_F32) {
+    F32Layer L = f32_layer(D);
+    const size_t smem = (size_t)(D->d + D->d_c + D->d_hr) * sizeof(float);
+    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+    f32_compress_append_kernel<<<T, 256, smem, as_stream(stream)>>>(
+        L, (const float*)h, (const float*)w->w_dkv, (const float*)w->w_kr, seq_idx, pos, (float*)cache->pool,
+        cache->num_blocks, cache->block_table, cache->max_blocks);
+    return check_launch();
+  }
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_compress_append(D, w, h, seq_idx, pos, T, cache, ws, ws_bytes, as_stream(stream));
+}
+
+mla_status_t mla_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos, int T,
+                          void* q_lat, void* q_rope, void* ws, size_t ws_bytes, void* stream) {
+  if (!desc_valid(D) || !w || !w->w_uq || !w->w_qr || !w->w_uk || (D->d_cq && !w->w_dq) || !h || !pos || T < 0 ||
+      !q_lat || !q_rope)
+    return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (D->dtype == MLA_F32) {
+    F32Layer L = f32_layer(D);
+    const int q_in = D->d_cq ? D->d_cq : D->d;
+    const size_t smem = (size_t)(D->d + q_in + D->n_h * D->d_h + D->n_h * D->d_hr) * sizeof(float);
+    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(f32_absorb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    f32_absorb_q_kernel<<<T, 256, smem, as_stream(stream)>>>(L, (const float*)h, (const float*)w->w_dq,
+                                                               (const float*)w->w_uq, (const float*)w->w_qr,
+                                                               (const float*)w->w_uk, pos, (float*)q_lat,
+                                                               (float*)q_rope);
+    return check_launch();
+  }
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_absorb_q(D, w, h, pos, T, q_lat, q_rope, ws, ws_bytes, as_stream(stream));
+}
+
+static mla_status_t f32_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
+                                  const mla_paged_cache* cache, const int32_t* kv_len, const int32_t* q_start,
+                                  int q_per_seq, int rows, void* ws, size_t ws_bytes, void* o_lat, float* lse,
+                                  cudaStream_t stream) {
+  const int max_len = cache->max_blocks * D->block_size;
+  if (!ws || ws_bytes < f32_attn_ws(D, rows, max_len)) return MLA_ERR_CAPACITY;
+  F32Layer L = f32_layer(D);
+  dim3 grid(rows, D->n_h);
+  f32_attn_kernel<<<grid, 128, 0, stream>>>(L, (const float*)q_lat, (const float*)q_rope, (const float*)cache->pool,
+                                            cache->num_blocks, cache->block_table, cache->max_blocks, kv_len,
+                                            q_start, q_per_seq, (float*)ws, max_len, (float*)o_lat, lse);
+  return check_launch();
+}
+
+mla_status_t mla_decode_attn(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
+                             const mla_paged_cache* cache, const int32_t* kv_len, int B, void* ws, size_t ws_bytes,
+                             int num_splits, void* o_lat, float* lse, void* stream) {
+  if (!desc_valid(D) || !q_lat || !q_rope || !cache_valid(cache) || !kv_len || B < 0 || num_splits < 0 || !o_lat)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (D->dtype == MLA_F32)
+    return f32_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, ws, ws_bytes, o_lat, lse,
+                         as_stream(stream));
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, ws, ws_bytes, num_splits, o_lat, lse,
+                      as_stream(stream));
+}
+
+mla_status_t mla_prefill_attn(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
+                              const mla_paged_cache* cache, const int32_t* q_start, int q_per_seq, int B, void* ws,
+                              size_t ws_bytes, void* o_lat, float* lse, void* stream) {
+  if (!desc_valid(D) || !q_lat || !q_rope || !cache_valid(cache) || !q_start || q_per_seq <= 0 || B < 0 || !o_lat)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  const long long rows = (long long)B * q_per_seq;
+  if (rows > (1 << 30)) return MLA_ERR_UNSUPPORTED;
+  if (D->dtype == MLA_F32)
+    return f32_attention(D, q_lat, q_rope, cache, nullptr, q_start, q_per_seq, (int)rows, ws, ws_bytes, o_lat, lse,
+                         as_stream(stream));
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_attention(D, q_lat, q_rope, cache, nullptr, q_start, q_per_seq, (int)rows, ws, ws_bytes, 1, o_lat, lse,
+                      as_stream(stream));
+}
+
+mla_status_t mla_out_proj(const mla_layer_desc* D, const mla_weights* w, const void* o_lat, int T, float* u, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (!desc_valid(D) || !w || !w->w_uv || !w->w_o || !o_lat || T < 0 || !u) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (D->dtype == MLA_F32) {
+    F32Layer L = f32_layer(D);
+    const size_t smem = (size_t)(D->n_h * D->d_c + D->n_h * D->d_h) * sizeof(float);
+    if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(f32_out_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    f32_out_proj_kernel<<<T, 256, smem, as_stream(stream)>>>(L, (const float*)o_lat, (const float*)w->w_uv,
+                                                               (const float*)w->w_o, u);
+    return check_launch();
+  }
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_out_proj(D, w, o_lat, T, u, ws, ws_bytes, as_stream(stream));
+}
+
+mla_status_t mla_get_last_error(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int code = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&code, g_error_code, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (code != 0) {
+    cudaMemcpyToSymbol(g_error_code, &zero, sizeof(int));
+    cudaMemcpyToSymbol(g_error_site, &zero, sizeof(int));
+    return code == ERR_TIMEOUT ? MLA_ERR_DEVICE_TIMEOUT : MLA_ERR_CAPACITY;
+  }
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // extern "C"

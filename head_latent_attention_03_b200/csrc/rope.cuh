@@ -1,0 +1,43 @@
+// rope.cuh — rotary frequencies of the decoupled RoPE carrier (q^R, k^R).
+//
+// DeepSeek-V2 explainer (adg.csdn.net) section 2.2.2: RoPE rides on extra
+// per-head queries q^R and one shared key k^R; section 3.1.3: YaRN (scale s,
+// alpha, beta over the original 4K window) is applied to that key.
+// Pair k of a d_h^R-wide vector turns by pos * theta_k with
+// theta_k = base^(-2k/d_h^R); with YaRN, pairs whose rotation count r_k over
+// the original window is below alpha are slowed by s, above beta kept, and
+// blended linearly in between ("NTK-by-parts").  Angles are formed in fp64:
+// at position 131072 an fp32 product pos * theta would be off by ~1e-2 rad.
+#pragma once
+
+#include <math.h>
+
+namespace mla {
+
+struct RopeParams {
+  double base, yarn_scale, yarn_alpha, yarn_beta;
+  int yarn_orig_ctx;
+};
+
+__host__ __device__ inline double rope_theta(const RopeParams& rp, int d_hr, int k) {
+  const double theta = pow(rp.base, -2.0 * (double)k / (double)d_hr);
+  if (rp.yarn_scale == 1.0) return theta;
+  const double turns = (double)rp.yarn_orig_ctx * theta / (2.0 * 3.14159265358979323846);
+  if (turns < rp.yarn_alpha) return theta / rp.yarn_scale;
+  if (turns > rp.yarn_beta) return theta;
+  const double g = (turns - rp.yarn_alpha) / (rp.yarn_beta - rp.yarn_alpha);
+  return (1.0 - g) * theta / rp.yarn_scale + g * theta;
+}
+
+__device__ inline void rope_cos_sin_theta(double theta, long long pos, float* c, float* s) {
+  double sd, cd;
+  sincos((double)pos * theta, &sd, &cd);
+  *c = (float)cd;
+  *s = (float)sd;
+}
+
+__device__ inline void rope_cos_sin(const RopeParams& rp, int d_hr, int k, long long pos, float* c, float* s) {
+  rope_cos_sin_theta(rope_theta(rp, d_hr, k), pos, c, s);
+}
+
+}  // namespace mla

@@ -1,0 +1,510 @@
+// tc_kernels.cuh — host side of the bf16 tensor-core path.
+//
+// Builds TMA descriptors over the caller's buffers, plans K splits and KV
+// splits from the SM count, carves the caller's workspace and launches the
+// GEMM / attention / finishing kernels on the caller's stream.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "rope.cuh"
+#include "tc_attn.cuh"
+#include "tc_gemm.cuh"
+
+namespace mla {
+
+// ---------------------------------------------------------------------------
+// device properties and TMA descriptor encoding
+// ---------------------------------------------------------------------------
+inline int num_sms() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 map: `outer` rows of `inner` elements, rows `row_bytes` apart,
+// box = box_outer rows x box_inner elements, 128-byte swizzle.
+inline bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                   uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The paged cache as a 3D map {row values, slot, block}; box = one page of
+// 64 slots x 64 values.  Block coordinates past num_blocks read zeros.
+inline bool map_cache(CUtensorMap* m, const void* pool, int num_blocks, int row) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)row, 64, (cuuint64_t)num_blocks};
+  cuuint64_t strides[2] = {(cuuint64_t)row * 2, (cuuint64_t)row * 2 * 64};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------------------
+// workspace carving
+// ---------------------------------------------------------------------------
+struct Carver {
+  uint8_t* base;
+  size_t cap, used = 0;
+  void* take(size_t bytes) {
+    used = (used + 255) & ~size_t(255);
+    void* p = base ? base + used : nullptr;
+    used += bytes;
+    return p;
+  }
+  bool ok() const { return used <= cap; }
+};
+
+// ---------------------------------------------------------------------------
+// GEMM planning and launch
+// ---------------------------------------------------------------------------
+struct GemmPlan {
+  int tn, n_tiles, splits, kcs;
+};
+
+inline int pick_tn(int T) { return T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256; }
+
+inline GemmPlan plan_gemm(int m_tiles, int Z, int T, int K) {
+  GemmPlan p;
+  p.tn = pick_tn(T);
+  p.n_tiles = (T + p.tn - 1) / p.tn;
+  const int kc = K / GEMM_BK;
+  const long long tiles = (long long)m_tiles * p.n_tiles * Z;
+  const int want = (int)std::max<long long>(1, (2LL * num_sms() + tiles - 1) / tiles);
+  const int cap_traffic = std::max(1, K / (8 * std::max(T, 1)));  // fp32 partials <= 1/4 of weight bytes
+  int s = std::min({want, cap_traffic, std::max(1, kc / 2)});
+  p.kcs = (kc + s - 1) / s;
+  p.splits = (kc + p.kcs - 1) / p.kcs;
+  return p;
+}
+
+template <int TN, bool A_MN>
+inline cudaError_t launch_gemm_t(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B, const GemmArgs& g,
+                                 dim3 grid, cudaStream_t st) {
+  auto kfn = gemm_bf16_kernel<TN, A_MN>;
+  constexpr int smem = GemmCfg<TN>::SMEM;
+  cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  kfn<<<grid, GEMM_THREADS, smem, st>>>(A0, A1, B, g);
+  return cudaGetLastError();
+}
+
+template <bool A_MN>
+inline cudaError_t launch_gemm_tn(int tn, const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B,
+                                  const GemmArgs& g, dim3 grid, cudaStream_t st) {
+  switch (tn) {
+    case 32: return launch_gemm_t<32, A_MN>(A0, A1, B, g, grid, st);
+    case 64: return launch_gemm_t<64, A_MN>(A0, A1, B, g, grid, st);
+    case 128: return launch_gemm_t<128, A_MN>(A0, A1, B, g, grid, st);
+    default: return launch_gemm_t<256, A_MN>(A0, A1, B, g, grid, st);
+  }
+}
+
+// One projection: out[ks][z][t][n] over two weight segments (rows0 of A0,
+// rows1 of A1), K contraction, Z batches.
+struct GemmCall {
+  const void* a0;
+  int rows0;
+  const void* a1;  // may be null
+  int rows1;
+  long long a_row_elems;  // row pitch of A in elements (K-major: K; MN-major: features)
+  bool a_mn;              // A stored [k][n] (n contiguous)
+  int a_mn_rows;          // MN-major: total K rows of the map (Z * K)
+  const void* x;
+  long long x_rows, x_row_elems;  // X map: x_rows rows of x_row_elems
+  int K, T, Z, a_z_rows, b_z_cols;
+};
+
+inline mla_status_t run_gemm(const GemmCall& c, float* out, long long out_z, long long out_t, long long out_split,
+                             const GemmPlan& p, cudaStream_t st) {
+  CUtensorMap A0, A1, B;
+  bool ok;
+  if (!c.a_mn) {
+    ok = map_2d(&A0, c.a0, (uint64_t)c.K, (uint64_t)c.rows0 * c.Z, (uint64_t)c.a_row_elems * 2, 64, 128);
+    ok = ok && map_2d(&A1, c.a1 ? c.a1 : c.a0, (uint64_t)c.K, (uint64_t)(c.a1 ? c.rows1 : c.rows0) * c.Z,
+                      (uint64_t)c.a_row_elems * 2, 64, 128);
+  } else {
+    ok = map_2d(&A0, c.a0, (uint64_t)c.rows0, (uint64_t)c.a_mn_rows, (uint64_t)c.a_row_elems * 2, 64, 64);
+    A1 = A0;
+  }
+  ok = ok && map_2d(&B, c.x, (uint64_t)c.x_row_elems, (uint64_t)c.x_rows, (uint64_t)c.x_row_elems * 2, 64,
+                    (uint32_t)p.tn);
+  if (!ok) return MLA_ERR_CUDA;
+  GemmArgs g;
+  g.k_chunks = c.K / GEMM_BK;
+  g.k_chunks_split = p.kcs;
+  g.n_tiles = p.n_tiles;
+  g.m_tiles0 = (c.rows0 + GEMM_BM - 1) / GEMM_BM;
+  g.n_out0 = c.rows0;
+  g.n_out1 = c.a1 ? c.rows1 : 0;
+  g.T = c.T;
+  g.a_z_rows = c.a_z_rows;
+  g.b_z_cols = c.b_z_cols;
+  g.out = out;
+  g.out_split = out_split;
+  g.out_z = out_z;
+  g.out_t = out_t;
+  const int m_tiles = g.m_tiles0 + (c.a1 ? (c.rows1 + GEMM_BM - 1) / GEMM_BM : 0);
+  dim3 grid(m_tiles, p.n_tiles * p.splits, c.Z);
+  const cudaError_t e = c.a_mn ? launch_gemm_tn<true>(p.tn, A0, A1, B, g, grid, st)
+                               : launch_gemm_tn<false>(p.tn, A0, A1, B, g, grid, st);
+  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+inline unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
+
+inline RopeParams rope_of(const mla_layer_desc* D) {
+  RopeParams r;
+  r.base = D->rope_base;
+  r.yarn_scale = D->yarn_scale;
+  r.yarn_alpha = D->yarn_alpha;
+  r.yarn_beta = D->yarn_beta;
+  r.yarn_orig_ctx = D->yarn_orig_ctx;
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// per-op workspace needs (same carving order as the ops below)
+// ---------------------------------------------------------------------------
+inline GemmPlan plan_compress(const mla_layer_desc* D, int T) {
+  return plan_gemm((D->d_c + 127) / 128 + (D->d_hr + 127) / 128, 1, T, D->d);
+}
+inline GemmPlan plan_q1(const mla_layer_desc* D, int T) { return plan_gemm((D->d_cq + 127) / 128, 1, T, D->d); }
+inline GemmPlan plan_q2(const mla_layer_desc* D, int T) {
+  const int q_in = D->d_cq ? D->d_cq : D->d;
+  return plan_gemm((D->n_h * D->d_h + 127) / 128 + (D->n_h * D->d_hr + 127) / 128, 1, T, q_in);
+}
+inline GemmPlan plan_q3(const mla_layer_desc* D, int T) { return plan_gemm(D->d_c / 128, D->n_h, T, D->d_h); }
+inline GemmPlan plan_o1(const mla_layer_desc* D, int T) { return plan_gemm((D->d_h + 127) / 128, D->n_h, T, D->d_c); }
+inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
+  return plan_gemm((D->d + 127) / 128, 1, T, D->n_h * D->d_h);
+}
+
+inline size_t ws_compress(const mla_layer_desc* D, int T) {
+  Carver c{nullptr, 0};
+  c.take((size_t)plan_compress(D, T).splits * T * (D->d_c + D->d_hr) * 4);
+  return c.used;
+}
+inline size_t ws_absorb(const mla_layer_desc* D, int T) {
+  Carver c{nullptr, 0};
+  const int nq = D->n_h * D->d_h;
+  if (D->d_cq) {
+    c.take((size_t)T * D->d_cq * 2);
+  }
+  c.take((size_t)T * nq * 2);
+  size_t part = 0;
+  if (D->d_cq) part = std::max(part, (size_t)plan_q1(D, T).splits * T * D->d_cq * 4);
+  part = std::max(part, (size_t)plan_q2(D, T).splits * T * (nq + D->n_h * D->d_hr) * 4);
+  part = std::max(part, (size_t)plan_q3(D, T).splits * D->n_h * T * D->d_c * 4);
+  c.take(part);
+  return c.used;
+}
+inline size_t ws_out(const mla_layer_desc* D, int T) {
+  Carver c{nullptr, 0};
+  c.take((size_t)T * D->n_h * D->d_h * 2);
+  size_t part = std::max((size_t)plan_o1(D, T).splits * D->n_h * T * D->d_h * 4,
+                         (size_t)plan_o2(D, T).splits * T * D->d * 4);
+  c.take(part);
+  return c.used;
+}
+
+inline int heads_per_cta(const mla_layer_desc* D) { return D->n_h == 16 ? 16 : 32; }
+
+struct AttnPlan {
+  int n_splits, span;
+};
+inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int requested) {
+  AttnPlan p;
+  const int groups = D->n_h / heads_per_cta(D);
+  const long long base = (long long)rows * groups;
+  int s = requested;
+  if (s <= 0) s = (int)std::max<long long>(1, (2LL * num_sms() + base - 1) / base);
+  s = std::max(1, std::min(s, (max_len + ATT_TILE - 1) / ATT_TILE));
+  const int per = (max_len + s - 1) / s;
+  p.span = (per + ATT_TILE - 1) / ATT_TILE * ATT_TILE;
+  p.n_splits = (max_len + p.span - 1) / p.span;
+  return p;
+}
+inline size_t ws_attn(const mla_layer_desc* D, int rows, int max_len, int n_splits) {
+  if (n_splits <= 1) return 0;
+  Carver c{nullptr, 0};
+  c.take((size_t)n_splits * rows * D->n_h * ATT_DC * 4);
+  c.take((size_t)n_splits * rows * D->n_h * 4);
+  return c.used;
+}
+
+}  // namespace mla
+
+using namespace mla;
+
+static size_t tc_workspace_size(const mla_layer_desc* D, int T, int B, int max_kv_len) {
+  size_t w = 0;
+  if (T > 0) w = std::max({ws_compress(D, T), ws_absorb(D, T), ws_out(D, T)});
+  if (B > 0 && max_kv_len > 0) {
+    const int max_len = (max_kv_len + 63) / 64 * 64;
+    const AttnPlan p = plan_attn(D, B, max_len, 0);
+    const int s = std::max(p.n_splits, std::min(16, (max_len + ATT_TILE - 1) / ATT_TILE));
+    w = std::max(w, ws_attn(D, B, max_len, s));
+  }
+  return w + 256;
+}
+
+static Carver carve(void* ws, size_t ws_bytes) {
+  uint8_t* b = reinterpret_cast<uint8_t*>(ws);
+  const uintptr_t a = (reinterpret_cast<uintptr_t>(b) + 255) & ~uintptr_t(255);
+  const size_t lost = b ? a - reinterpret_cast<uintptr_t>(b) : 0;
+  return Carver{b ? reinterpret_cast<uint8_t*>(a) : nullptr, ws_bytes > lost ? ws_bytes - lost : 0};
+}
+
+static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weights* w, const void* h,
+                                       const int32_t* seq_idx, const int32_t* pos, int T, mla_paged_cache* cache,
+                                       void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!aligned16(h) || !aligned16(w->w_dkv) || !aligned16(w->w_kr) || !aligned16(cache->pool))
+    return MLA_ERR_INVALID_ARG;
+  Carver cv = carve(ws, ws_bytes);
+  const int row = D->d_c + D->d_hr;
+  const GemmPlan p = plan_compress(D, T);
+  float* part = (float*)cv.take((size_t)p.splits * T * row * 4);
+  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  GemmCall c{};
+  c.a0 = w->w_dkv;
+  c.rows0 = D->d_c;
+  c.a1 = w->w_kr;
+  c.rows1 = D->d_hr;
+  c.a_row_elems = D->d;
+  c.x = h;
+  c.x_rows = T;
+  c.x_row_elems = D->d;
+  c.K = D->d;
+  c.T = T;
+  c.Z = 1;
+  mla_status_t s = run_gemm(c, part, 0, row, (long long)T * row, p, st);
+  if (s != MLA_OK) return s;
+  const long long n = (long long)T * row / 2;
+  finish_compress_kernel<<<blocks_for(n, 256), 256, 0, st>>>(
+      part, p.splits, (long long)T * row, T, D->d_c, D->d_hr, rope_of(D), seq_idx, pos,
+      (__nv_bfloat16*)cache->pool, cache->num_blocks, cache->block_table, cache->max_blocks, D->block_size);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos,
+                                int T, void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!aligned16(h) || !aligned16(w->w_uq) || !aligned16(w->w_qr) || !aligned16(w->w_uk) ||
+      (D->d_cq && !aligned16(w->w_dq)) || !aligned16(q_lat) || !aligned16(q_rope))
+    return MLA_ERR_INVALID_ARG;
+  Carver cv = carve(ws, ws_bytes);
+  const int nq = D->n_h * D->d_h, nr = D->n_h * D->d_hr;
+  const int q_in = D->d_cq ? D->d_cq : D->d;
+  __nv_bfloat16* cq = D->d_cq ? (__nv_bfloat16*)cv.take((size_t)T * D->d_cq * 2) : nullptr;
+  __nv_bfloat16* qc = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
+  const GemmPlan p1 = D->d_cq ? plan_q1(D, T) : GemmPlan{};
+  const GemmPlan p2 = plan_q2(D, T), p3 = plan_q3(D, T);
+  size_t part_bytes = (size_t)p2.splits * T * (nq + nr) * 4;
+  part_bytes = std::max(part_bytes, (size_t)p3.splits * D->n_h * T * D->d_c * 4);
+  if (D->d_cq) part_bytes = std::max(part_bytes, (size_t)p1.splits * T * D->d_cq * 4);
+  float* part = (float*)cv.take(part_bytes);
+  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  mla_status_t s;
+  const void* qsrc = h;
+  if (D->d_cq) {  // c^Q = W^DQ h   (eq 12)
+    GemmCall c{};
+    c.a0 = w->w_dq;
+    c.rows0 = D->d_cq;
+    c.a_row_elems = D->d;
+    c.x = h;
+    c.x_rows = T;
+    c.x_row_elems = D->d;
+    c.K = D->d;
+    c.T = T;
+    c.Z = 1;
+    if ((s = run_gemm(c, part, 0, D->d_cq, (long long)T * D->d_cq, p1, st)) != MLA_OK) return s;
+    const long long n = (long long)T * D->d_cq / 2;
+    finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p1.splits, (long long)T * D->d_cq, 1, T, D->d_cq, 0,
+                                                            D->d_cq, cq, 0, D->d_cq);
+    qsrc = cq;
+  }
+  {  // [q^C ; q^R] = [W^UQ ; W^QR] c^Q   (eq 13 + decoupled query), RoPE on q^R
+    GemmCall c{};
+    c.a0 = w->w_uq;
+    c.rows0 = nq;
+    c.a1 = w->w_qr;
+    c.rows1 = nr;
+    c.a_row_elems = q_in;
+    c.x = qsrc;
+    c.x_rows = T;
+    c.x_row_elems = q_in;
+    c.K = q_in;
+    c.T = T;
+    c.Z = 1;
+    if ((s = run_gemm(c, part, 0, nq + nr, (long long)T * (nq + nr), p2, st)) != MLA_OK) return s;
+    const long long n = (long long)T * (nq + nr) / 2;
+    finish_q_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p2.splits, (long long)T * (nq + nr), T, nq, D->n_h,
+                                                         D->d_hr, rope_of(D), pos, qc, (__nv_bfloat16*)q_rope);
+  }
+  {  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major
+    GemmCall c{};
+    c.a0 = w->w_uk;
+    c.rows0 = D->d_c;
+    c.a_row_elems = D->d_c;
+    c.a_mn = true;
+    c.a_mn_rows = D->n_h * D->d_h;
+    c.x = qc;
+    c.x_rows = T;
+    c.x_row_elems = nq;
+    c.K = D->d_h;
+    c.T = T;
+    c.Z = D->n_h;
+    c.a_z_rows = D->d_h;
+    c.b_z_cols = D->d_h;
+    // part[ks][head][t][c] ; q_lat[t][head][c]
+    if ((s = run_gemm(c, part, (long long)T * D->d_c, D->d_c, (long long)D->n_h * T * D->d_c, p3, st)) != MLA_OK)
+      return s;
+    const long long n = (long long)D->n_h * T * D->d_c / 2;
+    finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p3.splits, (long long)D->n_h * T * D->d_c, D->n_h,
+                                                            T, D->d_c, (long long)T * D->d_c, D->d_c,
+                                                            (__nv_bfloat16*)q_lat, D->d_c, (long long)D->n_h * D->d_c);
+  }
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, const void* o_lat, int T, float* u,
+                                void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!aligned16(o_lat) || !aligned16(w->w_uv) || !aligned16(w->w_o)) return MLA_ERR_INVALID_ARG;
+  Carver cv = carve(ws, ws_bytes);
+  const int nq = D->n_h * D->d_h;
+  __nv_bfloat16* o = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
+  const GemmPlan p1 = plan_o1(D, T), p2 = plan_o2(D, T);
+  float* part = (float*)cv.take(std::max((size_t)p1.splits * D->n_h * T * D->d_h * 4, (size_t)p2.splits * T * D->d * 4));
+  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  mla_status_t s;
+  {  // o_i = W^UV_i o_lat_i  (eq 11 absorbed): per head, A = W^UV_i [d_h, d_c]
+    GemmCall c{};
+    c.a0 = w->w_uv;
+    c.rows0 = D->d_h;
+    c.a_row_elems = D->d_c;
+    c.x = o_lat;
+    c.x_rows = T;
+    c.x_row_elems = (long long)D->n_h * D->d_c;
+    c.K = D->d_c;
+    c.T = T;
+    c.Z = D->n_h;
+    c.a_z_rows = D->d_h;
+    c.b_z_cols = D->d_c;
+    if ((s = run_gemm(c, part, (long long)T * D->d_h, D->d_h, (long long)D->n_h * T * D->d_h, p1, st)) != MLA_OK)
+      return s;
+    const long long n = (long long)D->n_h * T * D->d_h / 2;
+    finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p1.splits, (long long)D->n_h * T * D->d_h, D->n_h,
+                                                            T, D->d_h, (long long)T * D->d_h, D->d_h, o, D->d_h, nq);
+  }
+  {  // u = W^O o   (eq 8)
+    GemmCall c{};
+    c.a0 = w->w_o;
+    c.rows0 = D->d;
+    c.a_row_elems = nq;
+    c.x = o;
+    c.x_rows = T;
+    c.x_row_elems = nq;
+    c.K = nq;
+    c.T = T;
+    c.Z = 1;
+    if ((s = run_gemm(c, part, 0, D->d, (long long)T * D->d, p2, st)) != MLA_OK) return s;
+    const long long n = (long long)T * D->d / 2;
+    finish_f32_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p2.splits, (long long)T * D->d, T, D->d, u);
+  }
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <int H>
+static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, const CUtensorMap& mc, const AttnArgs& a,
+                               dim3 grid, cudaStream_t st) {
+  auto kfn = mla_attn_kernel<H>;
+  constexpr int smem = AttnCfg<H>::SMEM;
+  cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  kfn<<<grid, ATT_THREADS, smem, st>>>(mq, mr, mc, a);
+  return cudaGetLastError();
+}
+
+static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
+                                 const mla_paged_cache* cache, const int32_t* kv_len, const int32_t* q_start,
+                                 int q_per_seq, int rows, void* ws, size_t ws_bytes, int num_splits, void* o_lat,
+                                 float* lse, cudaStream_t st) {
+  if (!aligned16(q_lat) || !aligned16(q_rope) || !aligned16(cache->pool) || !aligned16(o_lat))
+    return MLA_ERR_INVALID_ARG;
+  const int H = heads_per_cta(D);
+  const int max_len = cache->max_blocks * 64;
+  const AttnPlan p = plan_attn(D, rows, max_len, kv_len ? num_splits : 1);
+  Carver cv = carve(ws, ws_bytes);
+  float* o_part = nullptr;
+  float* lse_part = nullptr;
+  if (p.n_splits > 1) {
+    o_part = (float*)cv.take((size_t)p.n_splits * rows * D->n_h * ATT_DC * 4);
+    lse_part = (float*)cv.take((size_t)p.n_splits * rows * D->n_h * 4);
+    if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  }
+  CUtensorMap mq, mr, mc;
+  bool ok = map_2d(&mq, q_lat, ATT_DC, (uint64_t)rows * D->n_h, ATT_DC * 2, 64, (uint32_t)H);
+  ok = ok && map_2d(&mr, q_rope, ATT_DR, (uint64_t)rows * D->n_h, ATT_DR * 2, 64, (uint32_t)H);
+  ok = ok && map_cache(&mc, cache->pool, cache->num_blocks, ATT_DC + ATT_DR);
+  if (!ok) return MLA_ERR_CUDA;
+  AttnArgs a;
+  a.n_h = D->n_h;
+  a.rows = rows;
+  a.q_per_seq = q_per_seq;
+  a.span = p.span;
+  a.n_splits = p.n_splits;
+  a.num_blocks = cache->num_blocks;
+  a.max_blocks = cache->max_blocks;
+  a.scale_log2 = (float)(D->attn_logit_factor / sqrt((double)(D->d_h + D->d_hr)) * 1.4426950408889634);
+  a.table = cache->block_table;
+  a.kv_len = kv_len;
+  a.q_start = q_start;
+  a.o_lat = (__nv_bfloat16*)o_lat;
+  a.lse = lse;
+  a.o_part = o_part;
+  a.lse_part = lse_part;
+  dim3 grid(p.n_splits, D->n_h / H, rows);
+  const cudaError_t e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
+  if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (p.n_splits > 1) {
+    mla_combine_kernel<<<rows * D->n_h, 128, 0, st>>>(o_part, lse_part, p.n_splits, rows, D->n_h,
+                                                      (__nv_bfloat16*)o_lat, lse);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return MLA_OK;
+}

@@ -71,7 +71,7 @@ class Workload:
     cfg_id: int
     dims: LayerDims
     batch: int
-    prior: str  # "fixed:<L>" or "uniform:<lo>:<hi>"
+    prior: str  # "fixed:<L>", "uniform:<lo>:<hi>" or "list:<L0>,<L1>,..."
     new_tokens: int = 1  # tokens appended per sequence (1 = decode)
     permute_pages: bool = False
     h_std: str = "unit"  # "unit" -> h ~ N(0,1); "fan_in" -> N(0, 1/d)
@@ -155,6 +155,10 @@ def gen_weights(w: Workload) -> Dict[str, Optional[np.ndarray]]:
 
 def prior_lengths(w: Workload) -> np.ndarray:
     kind, *args = w.prior.split(":")
+    if kind == "list":
+        vals = [int(v) for v in args[0].split(",")]
+        assert len(vals) == w.batch
+        return np.array(vals, dtype=np.int64)
     if kind == "fixed":
         return np.full(w.batch, int(args[0]), dtype=np.int64)
     lo, hi = int(args[0]), int(args[1])

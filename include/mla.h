@@ -1,0 +1,168 @@
+/*
+ * mla.h — C ABI of the B200 (sm_100a) Multi-head Latent Attention decode path.
+ *
+ * One MLA attention layer of DeepSeek-V2, in the absorbed inference form:
+ *   c^KV_t = W^DKV h_t                       (eq 9)
+ *   k^R_t  = RoPE_t(W^KR h_t)                (decoupled RoPE key, taken from h_t)
+ *   c^Q_t  = W^DQ h_t  (or h_t, no compression)   (eq 12)
+ *   q^C_t  = W^UQ c^Q_t                      (eq 13)
+ *   q^R_t  = RoPE_t(W^QR c^Q_t), per head
+ *   q_lat_{t,i} = (W^UK_i)^T q^C_{t,i}       (W^UK absorbed into the query)
+ *   s_j    = scale (q_lat_i . c^KV_j + q^R_i . k^R_j),  scale = factor / sqrt(d_h + d_h^R)
+ *   o_lat_i = sum_j softmax_j(s) c^KV_j      (eq 7 over the latent cache)
+ *   u_t    = W^O [W^UV_1 o_lat_1; ...; W^UV_nh o_lat_nh]   (eqs 8, 11; W^UV absorbed)
+ * Equations (1)-(13) as printed in the "DeepSeek-V2" reading notes
+ * (irregular6612.github.io), sections 2.1.1-2.1.2; the decoupled RoPE, the
+ * concatenated query/key and the absorption of W^UK and W^UV follow the
+ * DeepSeek-V2 explainer (adg.csdn.net), section 2.2.2; the cached row
+ * [c^KV ; k^R] of d_c + d_h^R values per token, shared by every head, is the
+ * explainer's section 2.2.2 cache formula.
+ *
+ * Conventions (all calls):
+ *  - Every tensor argument is a DEVICE pointer owned by the caller; structs
+ *    (mla_layer_desc, mla_weights, mla_paged_cache) live in HOST memory and
+ *    hold device pointers.  The library never allocates or frees device
+ *    memory; scratch comes from the caller's `ws` of at least
+ *    mla_workspace_size() bytes (256-byte aligned).
+ *  - Row-major layouts.  Weights are [out, in] (the y = W x convention).
+ *    Element type is float for MLA_F32 layers and bfloat16 for MLA_BF16
+ *    layers, except where a float type is written out (lse, u).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*).
+ *    Host-detectable errors return immediately and launch nothing.  Kernels
+ *    that detect a bad page id or give up a bounded wait record it in a
+ *    device error word read by mla_get_last_error().
+ *  - There is no CPU fallback and no dispatch to other devices: a shape the
+ *    kernels do not support returns MLA_ERR_UNSUPPORTED.
+ *  - Results are deterministic for fixed arguments (no atomics in reductions).
+ *
+ * Supported shapes.
+ *  MLA_F32 (exact fp32 SIMT kernels): d_hr even, block_size >= 1, any d, n_h,
+ *    d_h, d_c, d_cq.
+ *  MLA_BF16 (tcgen05 tensor-core kernels): block_size == 64, d_c == 512,
+ *    d_hr == 64, d_h % 64 == 0, d % 64 == 0, d_cq % 64 == 0, n_h in {16, 32,
+ *    64, 128}.
+ */
+#ifndef MLA_H
+#define MLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,     /* null pointer, non-positive size, bad desc field */
+  MLA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (shape / dtype) */
+  MLA_ERR_CAPACITY = 3,        /* workspace too small, page id out of range */
+  MLA_ERR_CUDA = 4,            /* a CUDA runtime call failed */
+  MLA_ERR_DEVICE_TIMEOUT = 5   /* a kernel gave up a bounded wait */
+} mla_status_t;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype_t;
+
+/* Layer description, in the pages' notation. */
+typedef struct {
+  int d;            /* model width (input h_t has d values) */
+  int n_h;          /* attention heads */
+  int d_h;          /* per-head dimension of q^C, k^C, v^C */
+  int d_c;          /* KV latent dimension (c^KV) */
+  int d_cq;         /* query latent dimension d_c'; 0 = queries read h directly */
+  int d_hr;         /* decoupled RoPE dimension d_h^R (q^R per head, shared k^R) */
+  int block_size;   /* tokens per cache page */
+  mla_dtype_t dtype;
+  double rope_base;          /* theta_k = rope_base^(-2k/d_hr) */
+  double yarn_scale;         /* s; 1 = plain RoPE */
+  int yarn_orig_ctx;         /* original context window of the YaRN blend */
+  double yarn_alpha, yarn_beta;
+  double attn_logit_factor;  /* multiplies every logit; 1 when YaRN is off */
+} mla_layer_desc;
+
+/* Projection matrices, [out, in] row-major, element type = desc.dtype.
+ *   w_dkv [d_c, d]            w_kr [d_hr, d]          w_dq [d_cq, d] (NULL if d_cq == 0)
+ *   w_uq  [n_h*d_h, q_in]     w_qr [n_h*d_hr, q_in]   (q_in = d_cq, or d when d_cq == 0)
+ *   w_uk  [n_h*d_h, d_c]      w_uv [n_h*d_h, d_c]     (head i = rows i*d_h .. i*d_h+d_h-1)
+ *   w_o   [d, n_h*d_h]                                                            */
+typedef struct {
+  const void *w_dkv, *w_kr, *w_dq, *w_uq, *w_qr, *w_uk, *w_uv, *w_o;
+} mla_weights;
+
+/* Paged latent cache: pool [num_blocks, block_size, d_c + d_hr]; token j of
+ * sequence b lives at pool[block_table[b*max_blocks + j/block_size]][j % block_size].
+ * Slots that no sequence has written may hold any bits (NaN included): the
+ * attention kernels never let them reach a result. */
+typedef struct {
+  void* pool;
+  int num_blocks;
+  const int32_t* block_table;  /* [B, max_blocks] int32 */
+  int max_blocks;
+} mla_paged_cache;
+
+/* Bytes of scratch that every call below needs for T tokens per projection
+ * call and B sequences of at most max_kv_len cached tokens per attention call
+ * (prefill: B sequences x q_per_seq queries count as B*q_per_seq rows). */
+size_t mla_workspace_size(const mla_layer_desc* desc, int T, int B, int max_kv_len);
+
+/* Compress and append T new tokens (eq 9 + decoupled RoPE key).
+ *   h       [T, d]        hidden states
+ *   seq_idx [T] int32     sequence of each token (row of block_table)
+ *   pos     [T] int32     position of each token; its page must already be
+ *                         in block_table (pos / block_size < max_blocks)
+ * Writes cache->pool rows [c^KV (d_c) | RoPE_pos(W^KR h) (d_hr)].
+ * A page id outside [0, num_blocks) sets MLA_ERR_CAPACITY in the device error
+ * word and the row is skipped. */
+mla_status_t mla_compress_append(const mla_layer_desc* desc, const mla_weights* w,
+                                 const void* h, const int32_t* seq_idx, const int32_t* pos, int T,
+                                 mla_paged_cache* cache, void* ws, size_t ws_bytes, void* stream);
+
+/* Absorbed queries of T tokens (eqs 12-13, decoupled RoPE query, W^UK folded in).
+ *   h      [T, d]; pos [T] int32
+ *   q_lat  [T, n_h, d_c]   out: (W^UK_i)^T W^UQ_i c^Q
+ *   q_rope [T, n_h, d_hr]  out: RoPE_pos(W^QR_i c^Q)                      */
+mla_status_t mla_absorb_q(const mla_layer_desc* desc, const mla_weights* w,
+                          const void* h, const int32_t* pos, int T,
+                          void* q_lat, void* q_rope, void* ws, size_t ws_bytes, void* stream);
+
+/* Decode attention over the latent cache, one query per sequence.
+ *   q_lat [B, n_h, d_c], q_rope [B, n_h, d_hr]
+ *   kv_len [B] int32     rows attended by sequence b (including the token just
+ *                        appended), 1 <= kv_len[b] <= max_blocks*block_size
+ *   num_splits           KV splits per sequence; 0 = chosen from the SM count
+ *   o_lat [B, n_h, d_c]  out: softmax-weighted sum of c^KV (desc dtype)
+ *   lse   [B, n_h] float out (may be NULL): natural-log sum of exp(s_j)      */
+mla_status_t mla_decode_attn(const mla_layer_desc* desc, const void* q_lat, const void* q_rope,
+                             const mla_paged_cache* cache, const int32_t* kv_len, int B,
+                             void* ws, size_t ws_bytes, int num_splits,
+                             void* o_lat, float* lse, void* stream);
+
+/* Causal attention of a chunk of q_per_seq new queries per sequence (chunked
+ * prefill, after mla_compress_append of the chunk).  Query q of sequence b
+ * sits at position q_start[b] + q and attends rows 0 .. q_start[b] + q.
+ *   q_lat [B*q_per_seq, n_h, d_c], q_rope [B*q_per_seq, n_h, d_hr]
+ *   o_lat [B*q_per_seq, n_h, d_c], lse [B*q_per_seq, n_h] float (may be NULL) */
+mla_status_t mla_prefill_attn(const mla_layer_desc* desc, const void* q_lat, const void* q_rope,
+                              const mla_paged_cache* cache, const int32_t* q_start, int q_per_seq, int B,
+                              void* ws, size_t ws_bytes, void* o_lat, float* lse, void* stream);
+
+/* Output projection (eq 8 with W^UV absorbed): u = W^O [W^UV_i o_lat_i]_i.
+ *   o_lat [T, n_h, d_c]; u [T, d] float                                     */
+mla_status_t mla_out_proj(const mla_layer_desc* desc, const mla_weights* w, const void* o_lat, int T,
+                          float* u, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device error word
+ * (MLA_ERR_CAPACITY for a bad page id, MLA_ERR_DEVICE_TIMEOUT for an
+ * abandoned wait) or MLA_ERR_CUDA if the stream reported a CUDA error. */
+mla_status_t mla_get_last_error(void* stream);
+
+/* Static string for a status code. */
+const char* mla_status_string(mla_status_t status);
+
+/* Library version, for the loader check: (major << 16) | minor. */
+int mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H */

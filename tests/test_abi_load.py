@@ -1,0 +1,58 @@
+"""The C-ABI library builds, loads and exports every symbol include/mla.h
+declares (no GPU needed: only host-side entry points are called)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from head_latent_attention_03_b200 import build, mla
+from head_latent_attention_03_b200.inputs import TINY, LITE, V2
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "mla.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("mla_compress_append", "mla_absorb_q", "mla_decode_attn", "mla_prefill_attn", "mla_out_proj",
+              "mla_workspace_size", "mla_get_last_error", "mla_status_string"):
+        assert f in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_host_only_entry_points(lib):
+    assert mla.version() >> 16 == 0
+    assert mla.status_string(0) == "ok"
+    assert "timed out" in mla.status_string(5)
+    for dims in (TINY, LITE, V2):
+        d = mla.layer_desc(dims)
+        assert mla.workspace_size(d, 64, 64, 8256) > 0
+
+
+def test_invalid_arguments_are_rejected_without_a_gpu(lib):
+    d = mla.layer_desc(V2)
+    w = mla.Weights()
+    cache = mla.PagedCache()
+    # null pointers: host validation returns before any CUDA call
+    code = mla.lib().mla_compress_append(ctypes.byref(d), ctypes.byref(w), None, None, None, 4,
+                                         ctypes.byref(cache), None, 0, None)
+    assert code == 1
+    bad = mla.layer_desc(V2)
+    bad.d_hr = 63  # odd RoPE width
+    assert mla.workspace_size(bad, 1, 1, 64) == 0

@@ -1,0 +1,203 @@
+"""CUDA path vs the fp64 oracle, through the C ABI, on seeded synthetic inputs.
+
+Each case runs the whole layer step on the GPU (compress_append -> absorb_q
+-> decode/prefill attention -> out_proj) and compares every stage with the
+oracle's own intermediates computed from the same generator inputs:
+the appended cache row, q_lat / q_rope, o_lat / lse and u.  Tolerances:
+fp32 layers max relative error 1e-4; bf16 layers RMS-relative 5e-3 and max
+absolute 2e-2 (tests/metrics.py).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from head_latent_attention_03_b200 import inputs as I
+from head_latent_attention_03_b200 import mla
+from head_latent_attention_03_b200.layer import MLALayer
+from oracle import mla_oracle as O
+from tests.metrics import assert_bf16, assert_fp32, rms_rel, max_abs
+
+pytestmark = pytest.mark.gpu
+
+W_CACHE = {}
+
+
+def weights_for(w):
+    key = (w.cfg_id, w.dims)
+    if key not in W_CACHE:
+        W_CACHE[key] = I.gen_weights(w)
+    return W_CACHE[key]
+
+
+def run_gpu(w, batch, num_splits=0):
+    weights = weights_for(w)
+    layer = MLALayer(w.dims, weights)
+    st = layer.upload(batch)
+    layer.step(st, num_splits=num_splits)
+    torch.cuda.synchronize()
+    code = mla.get_last_error()
+    assert code == 0, mla.status_string(code)
+    return layer, st
+
+
+def np32(t):
+    return t.float().cpu().numpy()
+
+
+def new_rows(st, batch):
+    D = batch.workload.dims
+    pool = np32(st.pool)
+    out = []
+    for b, L in enumerate(batch.prior_len):
+        for t in range(batch.workload.new_tokens):
+            p = int(L) + t
+            out.append(pool[batch.block_table[b, p // D.block_size], p % D.block_size])
+    return np.stack(out)
+
+
+def compare(name, g, r, dims):
+    if dims.dtype == "f32":
+        assert_fp32(g, r, name)
+    else:
+        assert_bf16(g, r, name)
+
+
+def check_decode(w, seqs=None, num_splits=0, batch=None):
+    batch = batch or I.gen_batch(w)
+    layer, st = run_gpu(w, batch, num_splits)
+    D = w.dims
+    seqs = list(range(len(batch.prior_len))) if seqs is None else seqs
+    ref = O.decode_batch(batch, weights_for(w), seqs=seqs, absorbed=True)
+    ref_un = O.decode_batch(batch, weights_for(w), seqs=seqs, absorbed=False)
+    rows = new_rows(st, batch)[seqs]
+    compare("cache row", rows, np.stack([r["row"] for r in ref]), D)
+    compare("q_lat", np32(st.q_lat)[seqs], np.stack([r["q_lat"] for r in ref]), D)
+    compare("q_rope", np32(st.q_rope)[seqs], np.stack([r["q_r"] for r in ref]), D)
+    compare("o_lat", np32(st.o_lat)[seqs], np.stack([r["o_lat"] for r in ref]), D)
+    lse_g, lse_r = np32(st.lse)[seqs], np.stack([r["lse"] for r in ref])
+    assert np.max(np.abs(lse_g - lse_r)) < (1e-4 if D.dtype == "f32" else 2e-2), np.max(np.abs(lse_g - lse_r))
+    compare("u", np32(st.u)[seqs], np.stack([r["u"] for r in ref_un]), D)
+    return batch, st
+
+
+# ----------------------------------------------------------------------------
+# small cases: every sequence checked, several tiles and a ragged tail
+# ----------------------------------------------------------------------------
+def test_tiny_fp32_step():
+    check_decode(I.WORKLOADS["tiny"])
+
+
+def test_tiny_fp32_prefill_chunk():
+    w = dataclasses.replace(I.WORKLOADS["tiny"], batch=2, prior="list:5,64", new_tokens=9)
+    batch = I.gen_batch(w)
+    layer, st = run_gpu(w, batch)
+    D = w.dims
+    W = weights_for(w)
+    rows_g = new_rows(st, batch)
+    for b in range(2):
+        L = int(batch.prior_len[b])
+        prior = O.gather_rows(batch.pool, batch.block_table[b], L, D.block_size)
+        new_r, outs = O.prefill_sequence(D, W, batch.h[b * 9:(b + 1) * 9], L, prior, range(9), absorbed=True)
+        assert_fp32(rows_g[b * 9:(b + 1) * 9], new_r, "rows")
+        for q in range(9):
+            r = b * 9 + q
+            assert_fp32(np32(st.o_lat)[r], outs[q]["o_lat"], f"o_lat {b},{q}")
+            assert_fp32(np32(st.u)[r], outs[q]["u"], f"u {b},{q}")
+
+
+LITE_SMALL = dataclasses.replace(I.WORKLOADS["lite"], name="lite_small", batch=4, prior="list:0,63,200,700")
+V2_SMALL = dataclasses.replace(I.WORKLOADS["v2"], name="v2_small", batch=3, prior="list:127,128,1000")
+YARN_SMALL = dataclasses.replace(I.WORKLOADS["long"], name="yarn_small", batch=2, prior="list:129,3000")
+
+
+@pytest.mark.parametrize("w", [LITE_SMALL, V2_SMALL, YARN_SMALL], ids=lambda w: w.name)
+def test_bf16_small(w):
+    check_decode(w)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 5])
+def test_split_count_invariance(splits):
+    w = dataclasses.replace(LITE_SMALL, prior="list:300,1500,900,64")
+    check_decode(w, num_splits=splits)
+
+
+def test_page_order_invariance():
+    # the same sequences on a permuted page table give bit-identical results
+    w = dataclasses.replace(LITE_SMALL, prior="list:300,1500,900,64")
+    b1 = I.gen_batch(w)
+    _, st1 = run_gpu(w, b1, 3)
+    u1, o1 = np32(st1.u), np32(st1.o_lat)
+    b2 = I.gen_batch(dataclasses.replace(w, permute_pages=True))
+    perm = np.random.default_rng(5).permutation(b1.pool.shape[0])
+    pool2 = np.full_like(b1.pool, np.nan)
+    table2 = b1.block_table.copy()
+    for b in range(table2.shape[0]):
+        for j in range(table2.shape[1]):
+            if table2[b, j] >= 0:
+                pool2[perm[b1.block_table[b, j]]] = b1.pool[b1.block_table[b, j]]
+                table2[b, j] = perm[b1.block_table[b, j]]
+    b2 = dataclasses.replace(b1, pool=pool2, block_table=table2)
+    _, st2 = run_gpu(w, b2, 3)
+    assert np.array_equal(np32(st2.o_lat), o1)
+    assert np.array_equal(np32(st2.u), u1)
+
+
+def test_single_row_returns_new_latent():
+    # kv_len = 1: softmax over one key is exactly 1, o_lat = the appended c^KV
+    w = dataclasses.replace(LITE_SMALL, batch=2, prior="list:0,0")
+    batch = I.gen_batch(w)
+    _, st = run_gpu(w, batch)
+    rows = new_rows(st, batch)
+    assert np.array_equal(np32(st.o_lat), np.broadcast_to(rows[:, None, :512], (2, 16, 512)))
+
+
+def test_bad_page_id_reports_capacity_error():
+    w = dataclasses.replace(LITE_SMALL, batch=2, prior="list:100,300")
+    batch = I.gen_batch(w)
+    batch.block_table[1, 2] = batch.pool.shape[0] + 7
+    layer = MLALayer(w.dims, weights_for(w))
+    st = layer.upload(batch)
+    layer.attend(st)
+    assert mla.get_last_error() == 3  # MLA_ERR_CAPACITY, no fault
+    assert mla.get_last_error() == 0  # cleared
+
+
+# ----------------------------------------------------------------------------
+# full-size workloads, in the launch configuration bench.py times; the oracle
+# checks a sample of sequences
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("name,seqs", [("lite", [0, 31]), ("v2", None)])
+def test_full_size_sampled(name, seqs):
+    w = I.WORKLOADS[name]
+    if seqs is None:
+        lens = I.prior_lengths(w)
+        seqs = [int(np.argmin(lens)), int(np.argmax(lens))]
+    check_decode(w, seqs=seqs)
+
+
+def test_long_context_sampled():
+    w = I.WORKLOADS["long"]
+    batch = I.gen_batch(w)
+    layer, st = run_gpu(w, batch)
+    ref = O.decode_batch(batch, weights_for(w), seqs=[3], absorbed=True)[0]
+    assert_bf16(np32(st.o_lat)[3], ref["o_lat"], "o_lat")
+    assert_bf16(np32(st.u)[3], ref["u"], "u")
+
+
+def test_prefill_sampled():
+    w = I.WORKLOADS["prefill"]
+    batch = I.gen_batch(w)
+    layer, st = run_gpu(w, batch)
+    D, W = w.dims, weights_for(w)
+    b, n = 5, w.new_tokens
+    L = int(batch.prior_len[b])
+    prior = O.gather_rows(batch.pool, batch.block_table[b], L, D.block_size)
+    qs = [0, 1, 63, 64, 1000, n - 1]
+    new_r, outs = O.prefill_sequence(D, W, batch.h[b * n:(b + 1) * n], L, prior, qs, absorbed=True)
+    assert_bf16(new_rows(st, batch)[b * n:(b + 1) * n], new_r, "rows")
+    for q in qs:
+        assert_bf16(np32(st.o_lat)[b * n + q], outs[q]["o_lat"], f"o_lat q={q}")
+        assert_bf16(np32(st.u)[b * n + q], outs[q]["u"], f"u q={q}")
