@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the MLA decode layer step on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload v2|lite|long|prefill] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path over one batch: compress_append ->
+absorb_q -> decode attention (+ LSE combine) -> out_proj, through the C ABI.
+Default workload: the DeepSeek-V2-shaped layer, decode batch 64 with cache
+lengths uniform in [1, 8192] on a randomly permuted page table.  Its cache
+(302 MB) and weights (298 MB) exceed the 126 MB L2, so no flush is needed
+between steps.  Under torchrun each rank runs an independent replica (the
+decode batch shards by sequence; no collective on the data path).
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+comparison) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode tokens/s (1 B200) and achieved % of HBM / bf16 tensor roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD_TEXT = {
+    "v2": "DeepSeek-V2-shaped MLA layer (d=5120, n_h=128, d_h=128, d_c=512, d_c'=1536, d_h^R=64), bf16, "
+          "decode batch 64, prior cache lengths uniform in [1,8192], block 64, permuted page table",
+    "lite": "DeepSeek-V2-Lite-shaped MLA layer (d=2048, n_h=16, d_h=128, d_c=512, d_h^R=64), bf16, "
+            "decode batch 32, 4096 prior tokens each, block 64",
+    "long": "V2-shaped MLA layer, bf16, decode batch 4 over 131072 prior tokens each, YaRN s=40, split-KV",
+    "prefill": "V2-shaped MLA layer, bf16, chunked prefill: 8 sequences x 4096 new tokens over 4096 cached",
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="mla_clocks_", suffix=".csv")
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                n += 1
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": n}
+
+
+def physical_gpu_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    if ids and all(v.isdigit() for v in ids) and local < len(ids):
+        return int(ids[local])
+    return local
+
+
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "head_latent_attention_03_b200", "csrc", "tc_attn.cuh")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "attn_dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# work accounting (algorithmic, per attention launch)
+# ---------------------------------------------------------------------------
+def attention_work(dims, kv_len, rows):
+    """Bytes that must move and FLOPs of one attention launch (absorbed form)."""
+    tok = int(sum(kv_len))
+    bytes_ = tok * dims.row * 2 + rows * dims.n_h * dims.row * 2 + rows * dims.n_h * dims.d_c * 2
+    flops = tok * 2 * dims.n_h * (2 * dims.d_c + dims.d_hr)
+    return bytes_, flops
+
+
+def cpu_oracle_baseline(w, seconds: float = 12.0):
+    """Time the fp64 oracle (un-absorbed form) on whole sequences of the workload
+    until `seconds` have passed; tokens/s = decoded tokens / time."""
+    import numpy as np
+    from head_latent_attention_03_b200 import inputs as I
+    from oracle import mla_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    W = I.gen_weights(w)
+    lens = I.prior_lengths(w)
+    order = list(range(w.batch))
+    done, t_total, toks = 0, 0.0, 0
+    for b in order:
+        batch = I.gen_batch(w, seqs=[b])
+        t0 = time.perf_counter()
+        if w.new_tokens == 1:
+            O.decode_batch(batch, W, absorbed=False)
+            toks += 1
+        else:
+            D = w.dims
+            prior = O.gather_rows(batch.pool, batch.block_table[0], int(batch.prior_len[0]), D.block_size)
+            O.prefill_sequence(D, W, batch.h[:1], int(batch.prior_len[0]), prior, [0], absorbed=False)
+            toks += 1
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total >= seconds:
+            break
+    sample = (f"{done} whole sequence(s) of the workload (cache lengths {[int(lens[b]) for b in order[:done]]}), "
+              f"fp64 un-absorbed oracle (eqs 9-11 then MHA), numpy BLAS")
+    return {"value": toks / t_total, "unit": "tokens/s", "cores": int(cores), "kind": "oracle", "sample": sample}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from head_latent_attention_03_b200 import build, inputs as I, mla
+    from head_latent_attention_03_b200.layer import MLALayer
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    w = I.WORKLOADS[args.workload]
+    W = I.gen_weights(w)
+    batch = I.gen_batch(w)
+    layer = MLALayer(w.dims, W, device=str(dev))
+    st = layer.upload(batch)
+    rows = st.h.shape[0]
+    kv = (batch.prior_len + 1) if w.new_tokens == 1 else None
+    if w.new_tokens == 1:
+        attn_bytes, attn_flops = attention_work(w.dims, kv, rows)
+    else:
+        per_q = [int(L) + q + 1 for L in batch.prior_len for q in range(w.new_tokens)]
+        attn_bytes, attn_flops = attention_work(w.dims, per_q, rows)
+    stream = torch.cuda.current_stream()
+
+    def step(ev_pair=None):
+        layer.compress_append(st)
+        layer.absorb_q(st)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        layer.attend(st)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+        layer.out_proj(st)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    code = mla.get_last_error()
+    if code != 0:
+        raise RuntimeError(f"device status after warm-up: {mla.status_string(code)}")
+
+    sampler = ClockSampler(physical_gpu_index(local))
+    if not args.profile_run:
+        sampler.start()
+        # keep the GPU busy while the sampler spins up so its samples fall under load
+        t_pre = time.time()
+        while time.time() - t_pre < 0.6:
+            step()
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = mla.launch_count()
+    e0.record(stream)
+    for k in range(args.steps):
+        step(attn_ev[k])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    n_launch = mla.launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if not args.profile_run else {"sm_mhz": None, "sm_max_mhz": None,
+                                                          "reasons": ["not sampled (profile run)"]}
+    code = mla.get_last_error()
+    if code != 0:
+        raise RuntimeError(f"device status after timed steps: {mla.status_string(code)}")
+    t_ms = e0.elapsed_time(e1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
+    t_all = torch.tensor([t_ms, attn_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
+    t_ms, attn_ms = float(t_all[0]), float(t_all[1])
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    h_host = st.h.cpu().pin_memory()
+    pos_host = st.pos.cpu().pin_memory()
+    seq_host = st.seq_idx.cpu().pin_memory()
+    kv_host = st.kv_len.cpu().pin_memory()
+    u_host = torch.empty(st.u.shape, dtype=st.u.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_host, pos_host, seq_host, kv_host))
+    d2h = u_host.numel() * u_host.element_size()
+
+    def e2e_step():
+        st.h.copy_(h_host, non_blocking=True)
+        st.pos.copy_(pos_host, non_blocking=True)
+        st.seq_idx.copy_(seq_host, non_blocking=True)
+        st.kv_len.copy_(kv_host, non_blocking=True)
+        layer.step(st)
+        u_host.copy_(st.u, non_blocking=True)
+
+    e2e_steps = 0 if args.profile_run else args.steps
+    for _ in range(3 if e2e_steps else 0):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = torch.tensor([max(f0.elapsed_time(f1), 1e-9)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
+        dist.barrier()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        hbm = float(peaks["hbm_gbs"])
+        tensor = float(peaks["bf16_tflops"])
+        achieved_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
+        achieved_tf = attn_flops / (attn_ms * 1e-3) / 1e12
+        t_hbm, t_tensor = attn_bytes / (hbm * 1e9), attn_flops / (tensor * 1e12)
+        bound = "hbm" if t_hbm >= t_tensor else "tensor"
+        traffic = committed_traffic(args.workload)
+        if bound == "hbm":
+            roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved_gbs / hbm, 4)}
+        else:
+            roof = {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": tensor, "unit": "TFLOP/s",
+                    "frac": round(achieved_tf / tensor, 4)}
+        roof.update({"traffic": traffic, "kernel": "mla_attn_kernel (+ mla_combine_kernel)",
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+                     "other_roof": {"hbm_frac": round(achieved_gbs / hbm, 4),
+                                    "tensor_frac": round(achieved_tf / tensor, 4),
+                                    "attn_bytes_per_launch": attn_bytes, "attn_flops_per_launch": attn_flops,
+                                    "attn_us": round(attn_ms * 1e3, 2)}})
+        value = world * rows * args.steps / (t_ms * 1e-3)
+        e2e_value = world * rows * e2e_steps / (float(t_e2e[0]) * 1e-3) if e2e_steps else None
+        out = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(t_ms / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1/fan_in) weights, N(0,1) hidden states and prior latents)",
+            "config": {"workload": WORKLOAD_TEXT[args.workload], "tokens_per_step_per_gpu": rows,
+                       "l2": "inputs exceed L2 (cache + weights > 126 MB), no flush",
+                       "parallelism": f"{world} independent replica(s), sequences sharded, no collective"},
+            "roofline": roof,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+            "e2e": {"value": round(e2e_value, 1) if e2e_value else None, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": int(n_launch),
+            "impl": "ours",
+        }
+        if world == 1 and not args.no_cpu_baseline and not args.profile_run:
+            out["cpu_baseline"] = cpu_oracle_baseline(w)
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    from head_latent_attention_03_b200 import inputs as I
+    from oracle import mla_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] or [os.cpu_count() or 1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    w = I.WORKLOADS[args.workload]
+    W = I.gen_weights(w)
+    lens = I.prior_lengths(w)
+    # each step decodes one whole sequence of the workload (its new token over
+    # its full cache), cycling through the batch in order
+    order = list(range(w.batch)) if w.new_tokens == 1 else [0]
+    batches = {}
+
+    def one(i):
+        b = order[i % len(order)]
+        if b not in batches:
+            batches[b] = I.gen_batch(w, seqs=[b])
+        bt = batches[b]
+        if w.new_tokens == 1:
+            O.decode_batch(bt, W, absorbed=False)
+        else:
+            D = w.dims
+            prior = O.gather_rows(bt.pool, bt.block_table[0], int(bt.prior_len[0]), D.block_size)
+            O.prefill_sequence(D, W, bt.h[:1], int(bt.prior_len[0]), prior, [0], absorbed=False)
+
+    for i in range(max(3, args.warmup)):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(max(3, args.warmup) + i)
+    t = time.perf_counter() - t0
+    value = args.steps / t
+    sample = (f"each step = one sequence's decode token over its whole cache (fp64 un-absorbed oracle), cycling "
+              f"the {len(order)} sequences of the workload in order")
+    out = {"metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": int(os.environ.get(
+        "WORLD_SIZE", "1")), "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[args.workload]}, "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": int(cores), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["v2", "lite", "long", "prefill"], default="v2")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="only the timed device steps (for ncu launch lists): no clock sampling, e2e or CPU leg")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -14,6 +14,13 @@
 
 namespace mla {
 
+// host-side count of kernel launches (mla_launch_count)
+inline unsigned long long& launch_counter() {
+  static unsigned long long n = 0;
+  return n;
+}
+#define MLA_COUNT_LAUNCH() (++::mla::launch_counter())
+
 // ---------------------------------------------------------------------------
 // device error word (read and cleared by mla_get_last_error)
 // ---------------------------------------------------------------------------

@@ -83,6 +83,8 @@ extern "C" {
 
 int mla_version(void) { return (kVersionMajor << 16) | kVersionMinor; }
 
+unsigned long long mla_launch_count(void) { return launch_counter(); }
+
 const char* mla_status_string(mla_status_t s) {
   switch (s) {
     case MLA_OK: return "ok";
@@ -114,6 +116,7 @@ mla_status_t mla_compress_append(const mla_layer_desc* D, const mla_weights* w, 
     F32Layer L = f32_layer(D);
     const size_t smem = (size_t)(D->d + D->d_c + D->d_hr) * sizeof(float);
     if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+    MLA_COUNT_LAUNCH();
     f32_compress_append_kernel<<<T, 256, smem, as_stream(stream)>>>(
         L, (const float*)h, (const float*)w->w_dkv, (const float*)w->w_kr, seq_idx, pos, (float*)cache->pool,
         cache->num_blocks, cache->block_table, cache->max_blocks);
@@ -136,6 +139,7 @@ mla_status_t mla_absorb_q(const mla_layer_desc* D, const mla_weights* w, const v
     if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(f32_absorb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    MLA_COUNT_LAUNCH();
     f32_absorb_q_kernel<<<T, 256, smem, as_stream(stream)>>>(L, (const float*)h, (const float*)w->w_dq,
                                                                (const float*)w->w_uq, (const float*)w->w_qr,
                                                                (const float*)w->w_uk, pos, (float*)q_lat,
@@ -154,6 +158,7 @@ static mla_status_t f32_attention(const mla_layer_desc* D, const void* q_lat, co
   if (!ws || ws_bytes < f32_attn_ws(D, rows, max_len)) return MLA_ERR_CAPACITY;
   F32Layer L = f32_layer(D);
   dim3 grid(rows, D->n_h);
+  MLA_COUNT_LAUNCH();
   f32_attn_kernel<<<grid, 128, 0, stream>>>(L, (const float*)q_lat, (const float*)q_rope, (const float*)cache->pool,
                                             cache->num_blocks, cache->block_table, cache->max_blocks, kv_len,
                                             q_start, q_per_seq, (float*)ws, max_len, (float*)o_lat, lse);
@@ -200,6 +205,7 @@ mla_status_t mla_out_proj(const mla_layer_desc* D, const mla_weights* w, const v
     if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(f32_out_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    MLA_COUNT_LAUNCH();
     f32_out_proj_kernel<<<T, 256, smem, as_stream(stream)>>>(L, (const float*)o_lat, (const float*)w->w_uv,
                                                                (const float*)w->w_o, u);
     return check_launch();

@@ -121,6 +121,7 @@ inline cudaError_t launch_gemm_t(const CUtensorMap& A0, const CUtensorMap& A1, c
   auto kfn = gemm_bf16_kernel<TN, A_MN>;
   constexpr int smem = GemmCfg<TN>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  MLA_COUNT_LAUNCH();
   kfn<<<grid, GEMM_THREADS, smem, st>>>(A0, A1, B, g);
   return cudaGetLastError();
 }
@@ -317,6 +318,7 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   mla_status_t s = run_gemm(c, part, 0, row, (long long)T * row, p, st);
   if (s != MLA_OK) return s;
   const long long n = (long long)T * row / 2;
+  MLA_COUNT_LAUNCH();
   finish_compress_kernel<<<blocks_for(n, 256), 256, 0, st>>>(
       part, p.splits, (long long)T * row, T, D->d_c, D->d_hr, rope_of(D), seq_idx, pos,
       (__nv_bfloat16*)cache->pool, cache->num_blocks, cache->block_table, cache->max_blocks, D->block_size);
@@ -355,6 +357,7 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.Z = 1;
     if ((s = run_gemm(c, part, 0, D->d_cq, (long long)T * D->d_cq, p1, st)) != MLA_OK) return s;
     const long long n = (long long)T * D->d_cq / 2;
+    MLA_COUNT_LAUNCH();
     finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p1.splits, (long long)T * D->d_cq, 1, T, D->d_cq, 0,
                                                             D->d_cq, cq, 0, D->d_cq);
     qsrc = cq;
@@ -374,6 +377,7 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.Z = 1;
     if ((s = run_gemm(c, part, 0, nq + nr, (long long)T * (nq + nr), p2, st)) != MLA_OK) return s;
     const long long n = (long long)T * (nq + nr) / 2;
+    MLA_COUNT_LAUNCH();
     finish_q_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p2.splits, (long long)T * (nq + nr), T, nq, D->n_h,
                                                          D->d_hr, rope_of(D), pos, qc, (__nv_bfloat16*)q_rope);
   }
@@ -396,6 +400,7 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     if ((s = run_gemm(c, part, (long long)T * D->d_c, D->d_c, (long long)D->n_h * T * D->d_c, p3, st)) != MLA_OK)
       return s;
     const long long n = (long long)D->n_h * T * D->d_c / 2;
+    MLA_COUNT_LAUNCH();
     finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p3.splits, (long long)D->n_h * T * D->d_c, D->n_h,
                                                             T, D->d_c, (long long)T * D->d_c, D->d_c,
                                                             (__nv_bfloat16*)q_lat, D->d_c, (long long)D->n_h * D->d_c);
@@ -429,6 +434,7 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
     if ((s = run_gemm(c, part, (long long)T * D->d_h, D->d_h, (long long)D->n_h * T * D->d_h, p1, st)) != MLA_OK)
       return s;
     const long long n = (long long)D->n_h * T * D->d_h / 2;
+    MLA_COUNT_LAUNCH();
     finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p1.splits, (long long)D->n_h * T * D->d_h, D->n_h,
                                                             T, D->d_h, (long long)T * D->d_h, D->d_h, o, D->d_h, nq);
   }
@@ -445,6 +451,7 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
     c.Z = 1;
     if ((s = run_gemm(c, part, 0, D->d, (long long)T * D->d, p2, st)) != MLA_OK) return s;
     const long long n = (long long)T * D->d / 2;
+    MLA_COUNT_LAUNCH();
     finish_f32_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p2.splits, (long long)T * D->d, T, D->d, u);
   }
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
@@ -456,6 +463,7 @@ static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, con
   auto kfn = mla_attn_kernel<H>;
   constexpr int smem = AttnCfg<H>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  MLA_COUNT_LAUNCH();
   kfn<<<grid, ATT_THREADS, smem, st>>>(mq, mr, mc, a);
   return cudaGetLastError();
 }
@@ -502,6 +510,7 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   const cudaError_t e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (p.n_splits > 1) {
+    MLA_COUNT_LAUNCH();
     mla_combine_kernel<<<rows * D->n_h, 128, 0, st>>>(o_part, lse_part, p.n_splits, rows, D->n_h,
                                                       (__nv_bfloat16*)o_lat, lse);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;

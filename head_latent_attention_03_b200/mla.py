@@ -46,6 +46,7 @@ _lib: Optional[ctypes.CDLL] = None
 
 _SIGS = {
     "mla_version": (ctypes.c_int, []),
+    "mla_launch_count": (ctypes.c_ulonglong, []),
     "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "mla_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(LayerDesc), ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "mla_compress_append": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
@@ -117,6 +118,11 @@ def paged_cache(pool, block_table) -> PagedCache:
 
 def version() -> int:
     return lib().mla_version()
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return lib().mla_launch_count()
 
 
 def status_string(code: int) -> str:

@@ -162,6 +162,10 @@ const char* mla_status_string(mla_status_t status);
 /* Library version, for the loader check: (major << 16) | minor. */
 int mla_version(void);
 
+/* Number of kernels this library has launched in this process (all devices,
+ * all streams), for accounting in benchmarks. */
+unsigned long long mla_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif
