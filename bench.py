@@ -113,9 +113,12 @@ def physical_gpu_index(local: int) -> int:
 
 
 def kernel_source_hash() -> str:
-    p = os.path.join(ROOT, "head_latent_attention_03_b200", "csrc", "tc_attn.cuh")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of every source the attention kernels are built from."""
+    h = hashlib.sha256()
+    for name in ("common.cuh", "tc_attn.cuh", "tc_attn2.cuh"):
+        with open(os.path.join(ROOT, "head_latent_attention_03_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def committed_traffic(workload: str):

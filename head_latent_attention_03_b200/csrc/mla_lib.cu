@@ -214,6 +214,17 @@ mla_status_t mla_out_proj(const mla_layer_desc* D, const mla_weights* w, const v
   return tc_out_proj(D, w, o_lat, T, u, ws, ws_bytes, as_stream(stream));
 }
 
+#ifdef MLA_TRACE
+// Trace builds only: copy the device trace buffer to `dst` (host) and clear it.
+int mla_trace_read(void* dst, size_t bytes) {
+  if (bytes > sizeof(g_trace)) bytes = sizeof(g_trace);
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(dst, g_trace, bytes) != cudaSuccess) return -1;
+  static unsigned long long zeros[MLA_TRACE_UNITS][MLA_TRACE_EVENTS][MLA_TRACE_TILES];
+  return cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros)) == cudaSuccess ? (int)bytes : -1;
+}
+#endif
+
 mla_status_t mla_get_last_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MLA_ERR_CUDA;
   int code = 0, zero = 0;

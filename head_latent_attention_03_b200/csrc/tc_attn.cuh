@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       uint32_t spins = 0;
       while (ok && jp < n_tiles) {
         bool prog = false;
-        if (jp < jq && mbar_try_wait(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1)) {
+        if (jp < jq && mbar_test(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1)) {
           tc_fence_after();
           const int pb = jp & 1;
           for (int m = 0; m < 4; ++m) {
@@ -239,21 +239,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         if (jq < n_tiles) {
           const int sb = jq & 1;
-          if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_try_wait(smem_u32(&s_free[sb]), ((jq >> 1) - 1) & 1);
+          if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_test(smem_u32(&s_free[sb]), ((jq >> 1) - 1) & 1);
           if (sbuf_ok) {
             bool ready;
             uint32_t ka;
             int qchunk;  // chunk of Q: 0..7 latent, 8 rope
             if (cq == 0) {
               const int rs = jq % C::NR;
-              ready = mbar_try_wait(smem_u32(&rope_full[rs]), (jq / C::NR) & 1);
+              ready = mbar_test(smem_u32(&rope_full[rs]), (jq / C::NR) & 1);
               ka = rope_base + rs * C::ROPE_SLOT;
               qchunk = 8;
             } else {
               const int c = cq - 1;
               const int li = jq * 4 + c / 2;
               const int s = li % C::NL;
-              ready = (c & 1) || mbar_try_wait(smem_u32(&lat_full[s]), (li / C::NL) & 1);
+              ready = (c & 1) || mbar_test(smem_u32(&lat_full[s]), (li / C::NL) & 1);
               ka = lat_base + s * C::LAT_SLOT + (c & 1) * 16384;
               qchunk = c;
             }
@@ -279,7 +279,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (prog) {
           t_idle = 0;
           spins = 0;
-        } else if ((++spins & 63u) == 0) {
+        } else if ((++spins & 63u) != 0) {
+          __nanosleep(64);  // back off: the barrier words are also updated by TMA and MMA completions
+        } else {
           if (*abort_flag) break;
           const uint64_t now = globaltimer_ns();
           if (t_idle == 0) {

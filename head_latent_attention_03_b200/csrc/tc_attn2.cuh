@@ -1,0 +1,534 @@
+// tc_attn2.cuh — latent-cache attention of 128-head layers on a CTA pair.
+//
+// Same arithmetic as tc_attn.cuh (absorbed MLA, DeepSeek-V2 explainer,
+// adg.csdn.net, section 2.2.2), laid out for n_h = 128: the two CTAs of a
+// cluster each own 64 heads and together issue tcgen05.mma.cta_group::2 with
+// the heads on M = 128.  Per 128-token tile (two cache pages, page r is
+// CTA r's "own" page):
+//   S[128 heads x 128 tok] = Q[128 x 576] . K^T    B split by page
+//   O[128 heads x 512]    += P[128 x 128] . V      B split by latent column:
+//                                                  CTA r holds columns 256i + [128r, 128r+128)
+// In the pair layout each CTA's TMEM holds its 64 heads folded over 128
+// lanes (lanes 64..127 carry the second half of the N columns), so S takes 64
+// columns and O 256: the fp32 O of all 128 heads (256 KB) no longer has to fit
+// one SM.  Q of 64 heads (72 KB) stays resident in shared memory.
+//
+// Cache data flow.  Each CTA loads its own page's row once, as a RoPE chunk
+// and four latent "pairs" (chunks 2k, 2k+1: 16 KB), and QK reads them.  PV
+// instruction (i, p) — latent columns of instruction i, tokens of page p —
+// reads pair slot k = 2i + p in BOTH CTAs (one descriptor for the pair): one
+// CTA already holds the right columns of its own page there, the other
+// overwrites its own (already multiplied) pair with the columns it needs from
+// the other page.  So every cached byte crosses into shared memory once per
+// CTA that needs it (104 KB per CTA per tile), and the eight 16 KB pair slots
+// keep two tiles in flight.  The cache is read through a 4D view
+// {column, slot, chunk, block} so that one TMA instruction fetches several
+// 64-column chunks of a page at once: per tile and CTA, one RoPE box, one
+// 8-chunk own-page box and two 2-chunk refill boxes.
+//
+// Warps (224 threads per CTA):
+//   0    own-page producer (RoPE chunk + the 8 latent chunks per tile)
+//   1    MMA issuer (leader CTA only, one thread) and TMEM owner (both CTAs)
+//   2-5  softmax: thread = (head, page half of the tile)
+//   6    other-page producer: refills the pair slots PV needs once QK is done
+//        with them; zeroes rows past kv_len in the last tile
+// TMA pair loads complete their bytes on the leader's barriers, for which the
+// leader alone posts the byte count; the only cluster-scope arrives are one
+// per CTA per tile from the softmax (S consumed, P written) and the last
+// tile's zeroing.  All waits are bounded.
+#pragma once
+
+#include "common.cuh"
+#include "tc_attn.cuh"
+
+namespace mla {
+
+struct PairCfg {
+  static constexpr int THREADS = 224;
+  static constexpr int Q_CHUNK = 64 * 128;        // 64 heads x 64 columns
+  static constexpr int Q_BYTES = 9 * Q_CHUNK;     // 72 KB
+  static constexpr int P_BYTES = 2 * 64 * 128;    // 64 heads x 128 tokens (two SW128 K atoms)
+  static constexpr int PAIR = 16384;              // one page x 2 latent chunks
+  static constexpr int ROPE = 8192;               // one page x 64 RoPE columns
+  static constexpr int NP = 8;                    // pair slots (two tiles)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_P = OFF_Q + Q_BYTES;
+  static constexpr int OFF_ROPE = OFF_P + P_BYTES;
+  static constexpr int OFF_PAIR = OFF_ROPE + ROPE;
+  static constexpr int OFF_BAR = OFF_PAIR + NP * PAIR;
+  static constexpr int N_BAR = 2 + 2 * NP + 1 + 1 + 2 + 2 + 1 + 2 + 1 + 1 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
+  static constexpr int OFF_RED = OFF_MISC + 16;
+  static constexpr int SMEM = OFF_RED + 3 * 128 * 4 + 1024;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(OFF_P % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_PAIR % 1024 == 0, "1 KB alignment");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+    mla_attn_pair_kernel(const __grid_constant__ CUtensorMap m_qlat, const __grid_constant__ CUtensorMap m_qrope,
+                         const __grid_constant__ CUtensorMap m_page1, const __grid_constant__ CUtensorMap m_page2,
+                         const __grid_constant__ CUtensorMap m_page8, const AttnArgs a) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  // Pair commits per tile: one qk_done per pair slot (QK has read it: the
+  // other CTA may refill it), s_full (S ready; the RoPE slot is free) and
+  // pv_done (the tile's pair slots are free, O is stable).  s_full and
+  // pv_done have one instance per tile parity so that a waiter is never two
+  // phases behind.
+  uint64_t* own_full = bar;                   // leader [2]: a tile's own latent chunks landed
+  uint64_t* oth_full = own_full + 2;          // leader [NP]: other-page refill landed
+  uint64_t* qk_done = oth_full + C::NP;       // both [NP]: pair commit once QK has read the slot
+  uint64_t* rope_full = qk_done + C::NP;      // leader
+  uint64_t* q_full = rope_full + 1;           // leader
+  uint64_t* s_full = q_full + 1;              // both [2]: pair commit after QK(j)
+  uint64_t* s_free = s_full + 2;              // leader [2]: one arrive per CTA
+  uint64_t* p_full = s_free + 2;              // leader: one arrive per CTA
+  uint64_t* pv_done = p_full + 1;             // both [2]: pair commit after PV(j)
+  uint64_t* last_ready = pv_done + 2;         // leader: both CTAs zeroed the last tile
+  uint64_t* grp_bar = last_ready + 1;         // local: 128 softmax threads
+  uint64_t* z_land = grp_bar + 1;             // local [2]: last tile's other-page refills
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [3][128]: tile max x2, final sums
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int split = blockIdx.x >> 1, r = blockIdx.z;
+  const int kv = att_kv_len(a, r);
+  const int seq = r / a.q_per_seq;
+  const int t_begin = split * a.span;
+  const int t_end = min(t_begin + a.span, kv);
+  const int n_tiles = t_end > t_begin ? (t_end - t_begin + ATT_TILE - 1) / ATT_TILE : 0;
+  const bool direct = a.n_splits == 1;
+  const int head0 = (int)rank * 64;
+  const int tunit = rank == 0 ? r * a.n_splits + split : -1;  // trace slot (leader only)
+  (void)tunit;
+
+  // both CTAs of the pair take the same early exits (same row and split)
+  if (kv < 1 || kv > a.max_blocks * 64) {
+    if (threadIdx.x == 0) record_error(ERR_CAPACITY, 501);
+    return;
+  }
+  if (n_tiles == 0) {
+    if (!direct)
+      for (int e = threadIdx.x; e < 64; e += blockDim.x)
+        a.lse_part[((long long)split * a.rows + r) * a.n_h + head0 + e] = -INFINITY;
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NP; ++i) {
+      mbar_init(&oth_full[i], 1);
+      mbar_init(&qk_done[i], 1);
+    }
+    mbar_init(rope_full, 1);
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&own_full[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 2);
+      mbar_init(&pv_done[i], 1);
+      mbar_init(&z_land[i], 1);
+    }
+    mbar_init(p_full, 2);
+    mbar_init(last_ready, 2);
+    mbar_init(grp_bar, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // peer barriers initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 0, 0);
+  const uint32_t tS = tmem;         // S buffers: columns [0,64) and [64,128)
+  const uint32_t tO = tmem + 128;   // O: columns [128,256) (d_c 0..255) and [256,384) (256..511)
+  const int* trow = a.table + (long long)seq * a.max_blocks;
+
+  // the last tile of a unit that reaches past kv_len: rows to zero before PV
+  auto needs_zero = [&](int j) -> bool { return t_begin + j * ATT_TILE + ATT_TILE > kv; };
+  auto page_block = [&](int page) -> int {
+    int b = a.num_blocks;  // past the sequence: TMA reads zeros
+    if (page * 64 < kv) {
+      b = trow[page];
+      if (b < 0 || b >= a.num_blocks) {
+        record_error(ERR_CAPACITY, 502);
+        b = a.num_blocks;
+      }
+    }
+    return b;
+  };
+  // pair slot of latent pair k of tile j, and how often that slot was used before
+  auto slot_of = [](int j, int k) -> int { return (4 * j + k) % C::NP; };
+  auto use_of = [](int j, int k) -> int { return (4 * j + k) / C::NP; };
+  // Pair k of a tile serves PV instruction k >> 1 over the tokens of page k & 1.
+  // The CTA whose own page is k & 1 keeps its own columns there; the other CTA
+  // refills the slot with columns 2*(2*(k>>1) + rank) .. +1 of page k & 1.
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ own-page producer
+    // Per tile two TMA instructions: the RoPE chunk (8 KB) and all eight
+    // latent chunks of the own page (64 KB, landing in the tile's four
+    // consecutive pair slots).  Few large boxes keep one issuing thread at
+    // full HBM rate.
+    if (elect_one()) {
+      tma_prefetch_desc(&m_page8);
+      if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
+      const uint32_t lq = mapa_shared(smem_u32(q_full), 0);
+      const int qrow = r * a.n_h + head0;
+      for (int c = 0; c < 8; ++c) tma_load_2d_pair(smem + C::OFF_Q + c * C::Q_CHUNK, &m_qlat, lq, c * 64, qrow);
+      tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
+      const int first_page = t_begin / 64 + (int)rank;
+      const uint32_t l_rope = mapa_shared(smem_u32(rope_full), 0);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int blk = page_block(first_page + 2 * j);
+        // the RoPE slot is free once QK(j-1) is done
+        if (j >= 1 && !mbar_wait(&s_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 503)) break;
+        if (rank == 0) mbar_expect_tx(rope_full, 2 * C::ROPE);
+        tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, 8, blk);
+        MLA_TRACE_EVENT(tunit, 1, j);
+        // the tile's four pair slots were last used by PV(j-2)
+        if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, 504)) break;
+        uint64_t* of = &own_full[j & 1];
+        if (rank == 0) mbar_expect_tx(of, 2 * 4 * C::PAIR);
+        tma_load_4d_pair(smem + C::OFF_PAIR + slot_of(j, 0) * C::PAIR, &m_page8, mapa_shared(smem_u32(of), 0), 0, 0,
+                         0, blk);
+        MLA_TRACE_EVENT(tunit, 2, j);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ other-page producer
+    for (int j = 0; j < n_tiles; ++j) {
+      const int tok = t_begin + j * ATT_TILE;
+      const bool zero = needs_zero(j);
+      bool ok = true;
+      if (lane == 0) {
+        int zk = 0;  // refills of this tile that land on z_land
+        for (int k = 0; k < 4 && ok; ++k) {
+          const int s = slot_of(j, k), u = use_of(j, k);
+          if ((k & 1) == (int)rank) continue;  // kept by this CTA
+          ok = mbar_wait(&qk_done[s], u & 1, abort_flag, 505);  // QK(j) has read this pair
+          if (!ok) break;
+          const int b = page_block(tok / 64 + (k & 1));
+          const int c0 = 2 * (2 * (k >> 1) + (int)rank);  // columns this CTA multiplies in instruction k >> 1
+          uint8_t* dst = smem + C::OFF_PAIR + s * C::PAIR;
+          if (!zero) {
+            if (rank == 0) mbar_expect_tx(&oth_full[s], C::PAIR);  // the peer's are posted by the MMA issuer
+            tma_load_4d_pair(dst, &m_page2, mapa_shared(smem_u32(&oth_full[s]), 0), 0, 0, c0, b);
+          } else {
+            mbar_expect_tx(&z_land[zk], C::PAIR);
+            tma_load_4d(dst, &m_page2, &z_land[zk], 0, 0, c0, b);
+            ++zk;
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      if (zero) {
+        // every pair this CTA presents to PV — refilled ones once landed, kept
+        // ones once QK is done with them — gets its rows past kv_len zeroed
+        const int first = kv - tok;
+        int zi = 0;
+        for (int k = 0; k < 4 && ok; ++k) {
+          const int s = slot_of(j, k);
+          const bool refilled = (k & 1) != (int)rank;
+          if (lane == 0)
+            ok = refilled ? mbar_wait(&z_land[zi], 0, abort_flag, 506)
+                          : mbar_wait(&qk_done[s], use_of(j, k) & 1, abort_flag, 507);
+          if (refilled) ++zi;
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          const int lo = max(0, first - 64 * (k & 1));  // first row of this page to clear
+          uint8_t* dst = smem + C::OFF_PAIR + s * C::PAIR;
+          for (int e = lo * 8 + lane; e < 64 * 8; e += 32) {
+            const int row = e >> 3, ch = e & 7;
+            *reinterpret_cast<uint4*>(dst + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(dst + 8192 + row * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive_cluster(mapa_shared(smem_u32(last_ready), 0));
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (rank == 0 && elect_one()) {
+      const uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t id_pv = idesc_bf16_f32(128, 256, false, true);
+      const uint32_t q_base = smem_u32(smem + C::OFF_Q);
+      const uint32_t rope_base = smem_u32(smem + C::OFF_ROPE);
+      const uint32_t pair0 = smem_u32(smem + C::OFF_PAIR);
+      const uint32_t p_base = smem_u32(smem + C::OFF_P);
+      // Byte counts of the refills the peer performs (pairs k = 0, 2) are
+      // posted here, each as soon as the slot's previous refill has been
+      // consumed by PV; the leader's own refills post theirs themselves.
+      auto post_peer_refills = [&](int j) {
+        if (j < n_tiles && !needs_zero(j))
+          for (int k = 0; k < 4; k += 2) mbar_expect_tx(&oth_full[slot_of(j, k)], C::PAIR);
+      };
+      post_peer_refills(0);
+      post_peer_refills(1);
+      bool ok = mbar_wait(q_full, 0, abort_flag, 511);
+      // Work is issued in batches (a tile's 32 latent QK MMAs at once, PV pair
+      // by pair): every barrier probe between MMAs costs issue slots.
+      int jq = 0, jp = 0, pv_k = 0;  // next QK tile, next PV tile, next pair of PV(jp)
+      bool sbuf_ok = false, rope_pending = false, p_ok = false;
+      uint64_t t_idle = 0;
+      uint32_t spins = 0;
+      while (ok && jp < n_tiles) {
+        bool prog = false;
+        // PV(jp) first: it frees the slots that later tiles' loads wait for
+        if (jp < jq) {
+          if (!p_ok) p_ok = mbar_test_cluster(smem_u32(p_full), jp & 1);
+          if (p_ok) {
+            const bool zero = needs_zero(jp);
+            while (pv_k < 4) {
+              const int s = slot_of(jp, pv_k), u = use_of(jp, pv_k);
+              const bool ready = zero ? mbar_test_cluster(smem_u32(last_ready), 0)
+                                      : mbar_test(smem_u32(&oth_full[s]), u & 1);
+              if (!ready) break;
+              if (pv_k == 0) MLA_TRACE_EVENT(tunit, 14, jp);
+              tc_fence_after();
+              const int i = pv_k >> 1, p = pv_k & 1;
+              const uint32_t pb = pair0 + s * C::PAIR;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = smem_desc(p_base + p * 8192 + kk * 32, 16, 1024, SW128);
+                const uint64_t bd = smem_desc(pb + kk * 2048, 8192, 1024, SW128);
+                mma_bf16_pair(tO + 128 * i, ad, bd, id_pv, (jp > 0 || p > 0 || kk > 0) ? 1u : 0u);
+              }
+              if ((pv_k & 1) == 0 && jp + 2 < n_tiles && !needs_zero(jp + 2))
+                mbar_expect_tx(&oth_full[slot_of(jp + 2, pv_k)], C::PAIR);
+              ++pv_k;
+              prog = true;
+            }
+            if (pv_k == 4) {
+              MLA_TRACE_EVENT(tunit, 5, jp);
+              mma_commit_pair(&pv_done[jp & 1]);
+              ++jp;
+              pv_k = 0;
+              p_ok = false;
+            }
+          }
+        }
+        if (jq < n_tiles) {
+          if (!rope_pending) {
+            if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_test_cluster(smem_u32(&s_free[jq & 1]), ((jq >> 1) - 1) & 1);
+            if (sbuf_ok && mbar_test(smem_u32(&own_full[jq & 1]), (jq >> 1) & 1)) {
+              MLA_TRACE_EVENT(tunit, 6, jq);
+              tc_fence_after();
+              // the 8 latent chunks, pair by pair; each pair's commit lets the
+              // other CTA refill that slot
+              for (int c = 0; c < 8; ++c) {
+                const uint32_t kb = pair0 + slot_of(jq, c >> 1) * C::PAIR + (c & 1) * 8192;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t ad = smem_desc(q_base + c * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
+                  const uint64_t bd = smem_desc(kb + kk * 32, 16, 1024, SW128);
+                  mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qk, (c | kk) != 0 ? 1u : 0u);
+                }
+                if (c & 1) mma_commit_pair(&qk_done[slot_of(jq, c >> 1)]);
+              }
+              rope_pending = true;
+              prog = true;
+            }
+          }
+          if (rope_pending && mbar_test(smem_u32(rope_full), jq & 1)) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = smem_desc(q_base + 8 * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
+              const uint64_t bd = smem_desc(rope_base + kk * 32, 16, 1024, SW128);
+              mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qk, 1u);
+            }
+            MLA_TRACE_EVENT(tunit, 7, jq);
+            mma_commit_pair(&s_full[jq & 1]);
+            ++jq;
+            rope_pending = false;
+            sbuf_ok = false;
+            prog = true;
+          }
+        }
+        if (prog) {
+          t_idle = 0;
+          spins = 0;
+        } else if ((++spins & 63u) != 0) {
+          __nanosleep(32);
+        } else {
+          if (*abort_flag) break;
+          const uint64_t now = globaltimer_ns();
+          if (t_idle == 0) {
+            t_idle = now;
+          } else if (now - t_idle > g_spin_limit_ns) {
+            record_error(ERR_TIMEOUT, 512);
+            *abort_flag = 1;
+            break;
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int q = warp & 3;
+    const int L = q * 32 + lane;     // TMEM lane
+    const int h = L & 63;            // head within this CTA
+    const int g = L >> 6;            // which page of the tile this thread's scores cover
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t l_sfree[2] = {mapa_shared(smem_u32(&s_free[0]), 0), mapa_shared(smem_u32(&s_free[1]), 0)};
+    const uint32_t l_pfull = mapa_shared(smem_u32(p_full), 0);
+    uint32_t gphase = 0;
+    auto group_sync = [&](int site) -> bool {
+      mbar_arrive(grp_bar);
+      const bool ok2 = mbar_wait(grp_bar, gphase & 1, abort_flag, site);
+      ++gphase;
+      return ok2;
+    };
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, 521)) {
+        ok = false;
+        break;
+      }
+      if (L == 0) MLA_TRACE_EVENT(tunit, 8, j);
+      tc_fence_after();
+      float s[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32<16>(tS + (j & 1) * 64 + c * 16 + lane_off, s + 16 * c);
+      tmem_wait_ld();
+      tc_fence_before();
+      const int tok0 = t_begin + j * ATT_TILE + 64 * g;
+      const int nvalid = min(64, max(0, t_end - tok0));
+      float pmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        s[c] = c < nvalid ? s[c] * a.scale_log2 : -INFINITY;
+        pmax = fmaxf(pmax, s[c]);
+      }
+      float* rb = red + (j & 1) * 128;
+      rb[L] = pmax;
+      if (!group_sync(522)) {
+        ok = false;
+        break;
+      }
+      // every thread's TMEM reads of S(j) are complete: release the buffer
+      if (L == 0) {
+        if (rank == 0)
+          mbar_arrive(&s_free[j & 1]);
+        else
+          mbar_arrive_cluster(l_sfree[j & 1]);
+      }
+      const float m_new = fmaxf(m_run, fmaxf(pmax, rb[L ^ 64]));
+      if (j >= 1) {
+        // PV(j-1) complete: the P buffer is free and O is stable
+        if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 523)) {
+          ok = false;
+          break;
+        }
+        if (L == 0) MLA_TRACE_EVENT(tunit, 9, j - 1);
+        tc_fence_after();
+      }
+      const bool grow = __any_sync(0xffffffffu, m_new > m_run + ATT_RESCALE_LOG2);
+      if (j == 0) {
+        m_run = m_new;
+      } else if (grow) {
+        const float alpha = exp2_approx(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 16) {
+          float o[16];
+          tmem_ld32<16>(tO + c + lane_off, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o[e] *= alpha;
+          tmem_st32<16>(tO + c + lane_off, o);
+        }
+        tmem_wait_st();
+      }
+      uint8_t* prow = smem + C::OFF_P + g * 8192 + h * 128;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = exp2_approx(s[8 * cc + 2 * e] - m_run);
+          const float p1 = exp2_approx(s[8 * cc + 2 * e + 1] - m_run);
+          l_run += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      if (!group_sync(526)) {
+        ok = false;
+        break;
+      }
+      if (L == 0) {
+        if (rank == 0)
+          mbar_arrive(p_full);
+        else
+          mbar_arrive_cluster(l_pfull);
+        MLA_TRACE_EVENT(tunit, 10, j);
+      }
+    }
+    // ------------------------------------------------------------ epilogue
+    float* lred = red + 256;
+    lred[L] = l_run;
+    ok = group_sync(524) && ok;
+    const float l_tot = l_run + lred[L ^ 64];
+    const int last = n_tiles - 1;
+    ok = ok && mbar_wait(&pv_done[last & 1], (last >> 1) & 1, abort_flag, 525);
+    tc_fence_after();
+    const float inv_l = 1.f / l_tot;
+    const long long ob = ((long long)r * a.n_h + head0 + h) * ATT_DC;
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 16) {
+      float o[16];
+      tmem_ld32<16>(tO + c + lane_off, o);
+      tmem_wait_ld();
+      if (!ok) continue;
+      // TMEM column c of this lane: latent index 256*(c/128) + 128*g + c%128
+      const int d = 256 * (c >> 7) + 128 * g + (c & 127);
+      if (direct) {
+        uint4 v0 = make_uint4(pack_bf16(o[0] * inv_l, o[1] * inv_l), pack_bf16(o[2] * inv_l, o[3] * inv_l),
+                              pack_bf16(o[4] * inv_l, o[5] * inv_l), pack_bf16(o[6] * inv_l, o[7] * inv_l));
+        uint4 v1 = make_uint4(pack_bf16(o[8] * inv_l, o[9] * inv_l), pack_bf16(o[10] * inv_l, o[11] * inv_l),
+                              pack_bf16(o[12] * inv_l, o[13] * inv_l), pack_bf16(o[14] * inv_l, o[15] * inv_l));
+        uint4* dst = reinterpret_cast<uint4*>(a.o_lat + ob + d);
+        dst[0] = v0;
+        dst[1] = v1;
+      } else {
+        float4* dst = reinterpret_cast<float4*>(a.o_part + (long long)split * a.rows * a.n_h * ATT_DC + ob + d);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_float4(o[4 * e] * inv_l, o[4 * e + 1] * inv_l, o[4 * e + 2] * inv_l, o[4 * e + 3] * inv_l);
+      }
+    }
+    if (ok && g == 0) {
+      const float lse = (m_run + log2f(l_tot)) * 0.69314718055994531f;
+      const long long li = (long long)r * a.n_h + head0 + h;
+      if (direct) {
+        if (a.lse) a.lse[li] = lse;
+      } else {
+        a.lse_part[(long long)split * a.rows * a.n_h + li] = lse;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 11, 0);
+  cluster_sync_all();  // the peer's MMAs, TMA signals and arrives are done
+  if (warp == 1) tmem_dealloc_pair(tmem, C::TMEM_COLS);
+}
+
+}  // namespace mla

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "rope.cuh"
 #include "tc_attn.cuh"
+#include "tc_attn2.cuh"
 #include "tc_gemm.cuh"
 
 namespace mla {
@@ -71,6 +72,22 @@ inline bool map_cache(CUtensorMap* m, const void* pool, int num_blocks, int row)
   cuuint32_t box[3] = {64, 64, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The paged cache as a 4D map {column in chunk, slot, 64-column chunk, block}
+// (the chunk stride, 128 bytes, is smaller than the slot stride): a box of
+// `chunks` chunks of one page lands chunk-major, 8 KB per chunk, so one TMA
+// instruction moves up to a whole page.
+inline bool map_cache_chunks(CUtensorMap* m, const void* pool, int num_blocks, int row, int chunks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, 64, (cuuint64_t)(row / 64), (cuuint64_t)num_blocks};
+  cuuint64_t strides[3] = {(cuuint64_t)row * 2, 128, (cuuint64_t)row * 2 * 64};
+  cuuint32_t box[4] = {64, 64, (cuuint32_t)chunks, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(pool), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -246,16 +263,21 @@ inline size_t ws_out(const mla_layer_desc* D, int T) {
 }
 
 inline int heads_per_cta(const mla_layer_desc* D) { return D->n_h == 16 ? 16 : 32; }
+// 128-head layers run on CTA pairs (tc_attn2.cuh), one pair per (row, split)
+inline bool use_pair_kernel(const mla_layer_desc* D) { return D->n_h == 128; }
 
 struct AttnPlan {
   int n_splits, span;
 };
 inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int requested) {
   AttnPlan p;
-  const int groups = D->n_h / heads_per_cta(D);
+  // work units in flight per wave: one per SM, or one per SM pair
+  const bool pair = use_pair_kernel(D);
+  const int groups = pair ? 1 : D->n_h / heads_per_cta(D);
   const long long base = (long long)rows * groups;
+  const long long target = pair ? 2LL * (num_sms() / 2) : 2LL * num_sms();
   int s = requested;
-  if (s <= 0) s = (int)std::max<long long>(1, (2LL * num_sms() + base - 1) / base);
+  if (s <= 0) s = (int)std::max<long long>(1, (target + base - 1) / base);
   s = std::max(1, std::min(s, (max_len + ATT_TILE - 1) / ATT_TILE));
   const int per = (max_len + s - 1) / s;
   p.span = (per + ATT_TILE - 1) / ATT_TILE * ATT_TILE;
@@ -485,9 +507,11 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
     lse_part = (float*)cv.take((size_t)p.n_splits * rows * D->n_h * 4);
     if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   }
+  const bool pair = use_pair_kernel(D);
+  const uint32_t q_box = pair ? 64u : (uint32_t)H;  // query rows per CTA
   CUtensorMap mq, mr, mc;
-  bool ok = map_2d(&mq, q_lat, ATT_DC, (uint64_t)rows * D->n_h, ATT_DC * 2, 64, (uint32_t)H);
-  ok = ok && map_2d(&mr, q_rope, ATT_DR, (uint64_t)rows * D->n_h, ATT_DR * 2, 64, (uint32_t)H);
+  bool ok = map_2d(&mq, q_lat, ATT_DC, (uint64_t)rows * D->n_h, ATT_DC * 2, 64, q_box);
+  ok = ok && map_2d(&mr, q_rope, ATT_DR, (uint64_t)rows * D->n_h, ATT_DR * 2, 64, q_box);
   ok = ok && map_cache(&mc, cache->pool, cache->num_blocks, ATT_DC + ATT_DR);
   if (!ok) return MLA_ERR_CUDA;
   AttnArgs a;
@@ -506,8 +530,22 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   a.lse = lse;
   a.o_part = o_part;
   a.lse_part = lse_part;
-  dim3 grid(p.n_splits, D->n_h / H, rows);
-  const cudaError_t e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
+  cudaError_t e;
+  if (pair) {
+    CUtensorMap m1, m2, m8;
+    if (!map_cache_chunks(&m1, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 1) ||
+        !map_cache_chunks(&m2, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 2) ||
+        !map_cache_chunks(&m8, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 8))
+      return MLA_ERR_CUDA;
+    dim3 grid(2 * p.n_splits, 1, rows);
+    cudaFuncSetAttribute(mla_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
+    MLA_COUNT_LAUNCH();
+    mla_attn_pair_kernel<<<grid, PairCfg::THREADS, PairCfg::SMEM, st>>>(mq, mr, m1, m2, m8, a);
+    e = cudaGetLastError();
+  } else {
+    dim3 grid(p.n_splits, D->n_h / H, rows);
+    e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
+  }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (p.n_splits > 1) {
     MLA_COUNT_LAUNCH();
