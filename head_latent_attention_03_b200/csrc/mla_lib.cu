@@ -79,6 +79,35 @@ size_t f32_attn_ws(const mla_layer_desc* D, int rows, int max_len) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for mla_decode_attn_noalloc: a fixed device array owned by this
+// library instead of a caller workspace.  Every device that loads the library
+// holds it until the process exits.  Host code may not use the symbol itself
+// as a device address; the address is looked up per device.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = 32u << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device, with that device current).  nullptr if the lookup fails.
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
 extern "C" {
 
 int mla_version(void) { return (kVersionMajor << 16) | kVersionMinor; }
@@ -177,6 +206,36 @@ mla_status_t mla_decode_attn(const mla_layer_desc* D, const void* q_lat, const v
   if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
   return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, ws, ws_bytes, num_splits, o_lat, lse,
                       as_stream(stream));
+}
+
+mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
+                                     const mla_paged_cache* cache, const int32_t* kv_len, int B, int num_splits,
+                                     void* o_lat, float* lse, void* stream) {
+  if (!desc_valid(D) || !q_lat || !q_rope || !cache_valid(cache) || !kv_len || B < 0 || num_splits < 0 || !o_lat)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  void* scratch = noalloc_scratch();
+  if (!scratch) return MLA_ERR_CUDA;
+  // Every partial the kernels read back is written first in the same call,
+  // so the array needs no clearing between calls.
+  const int max_len = cache->max_blocks * D->block_size;
+  if (D->dtype == MLA_F32) {
+    if (f32_attn_ws(D, B, max_len) > kNoAllocScratchBytes) return MLA_ERR_CAPACITY;
+    return f32_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, scratch, kNoAllocScratchBytes, o_lat, lse,
+                         as_stream(stream));
+  }
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  int splits = num_splits;
+  if (splits == 0) {
+    // the automatic split count, reduced until the partials fit the array
+    splits = plan_attn(D, B, max_len, 0).n_splits;
+    while (splits > 1 && ws_attn(D, B, max_len, plan_attn(D, B, max_len, splits).n_splits) + 512 > kNoAllocScratchBytes)
+      --splits;
+  } else if (ws_attn(D, B, max_len, plan_attn(D, B, max_len, splits).n_splits) + 512 > kNoAllocScratchBytes) {
+    return MLA_ERR_CAPACITY;
+  }
+  return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, scratch, kNoAllocScratchBytes, splits, o_lat,
+                      lse, as_stream(stream));
 }
 
 mla_status_t mla_prefill_attn(const mla_layer_desc* D, const void* q_lat, const void* q_rope,

@@ -60,6 +60,9 @@ _SIGS = {
                                        ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                        ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p]),
+    "mla_decode_attn_noalloc": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "mla_prefill_attn": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
@@ -150,6 +153,14 @@ def decode_attn(desc, q_lat, q_rope, cache: PagedCache, kv_len, ws, o_lat, lse=N
         ctypes.byref(desc), _ptr(q_lat), _ptr(q_rope), ctypes.byref(cache), _ptr(kv_len), kv_len.shape[0],
         _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, num_splits, _ptr(o_lat), _ptr(lse),
         _stream(stream)))
+
+
+def decode_attn_noalloc(desc, q_lat, q_rope, cache: PagedCache, kv_len, o_lat, lse=None, num_splits=0, stream=None):
+    """mla_decode_attn with the library's own fixed scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    _check("mla_decode_attn_noalloc", lib().mla_decode_attn_noalloc(
+        ctypes.byref(desc), _ptr(q_lat), _ptr(q_rope), ctypes.byref(cache), _ptr(kv_len), kv_len.shape[0],
+        num_splits, _ptr(o_lat), _ptr(lse), _stream(stream)))
 
 
 def prefill_attn(desc, q_lat, q_rope, cache: PagedCache, q_start, q_per_seq, ws, o_lat, lse=None, stream=None):

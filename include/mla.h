@@ -137,6 +137,31 @@ mla_status_t mla_decode_attn(const mla_layer_desc* desc, const void* q_lat, cons
                              void* ws, size_t ws_bytes, int num_splits,
                              void* o_lat, float* lse, void* stream);
 
+/* mla_decode_attn without a caller workspace (the pages have no counterpart:
+ * this is a deployment variant, not part of the method).
+ * For callers that cannot allocate device memory at call time — code running
+ * inside a region that forbids allocation (a captured or replayed command
+ * stream, a real-time serving loop whose memory was fixed at start-up, a
+ * plug-in that may not touch the host framework's allocator) and that has no
+ * spare buffer to lend as workspace.
+ * Same arguments and results as mla_decode_attn, minus the workspace.  The
+ * split partials live in a library-owned device array of 32 MiB
+ * (every device that loads the library holds it until the process exits);
+ * with num_splits == 0 the automatic split count is lowered until the
+ * partials fit, an explicit num_splits whose partials need more than 32 MiB
+ * (num_splits * B * n_h * 2052 bytes, bf16 layers) returns MLA_ERR_CAPACITY,
+ * as does an fp32 layer whose score scratch (B * n_h * max_blocks *
+ * block_size * 4 bytes) exceeds it.  No device memory is allocated or freed.
+ * The first call on a device looks up the array's address on that device (a
+ * host-side runtime query): make that first call before any stream capture.
+ * All calls share the one array and every partial is written before it is
+ * read, so nothing needs clearing; calls that may run concurrently on the
+ * GPU (different streams, or two devices' work racing on one device) race on
+ * it and must be serialised by the caller. */
+mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* desc, const void* q_lat, const void* q_rope,
+                                     const mla_paged_cache* cache, const int32_t* kv_len, int B, int num_splits,
+                                     void* o_lat, float* lse, void* stream);
+
 /* Causal attention of a chunk of q_per_seq new queries per sequence (chunked
  * prefill, after mla_compress_append of the chunk).  Query q of sequence b
  * sits at position q_start[b] + q and attends rows 0 .. q_start[b] + q.
