@@ -164,6 +164,12 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // ---------------------------------------------------------------------------
 // TMA tiled loads into the issuing CTA's shared memory
 // ---------------------------------------------------------------------------
+// Bulk prefetch of a contiguous global range into L2 (no shared memory, no
+// completion): address and size multiples of 16 bytes.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }

@@ -225,17 +225,20 @@ mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* D, const void* q_lat,
                          as_stream(stream));
   }
   if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
-  int splits = num_splits;
-  if (splits == 0) {
-    // the automatic split count, reduced until the partials fit the array
-    splits = plan_attn(D, B, max_len, 0).n_splits;
-    while (splits > 1 && ws_attn(D, B, max_len, plan_attn(D, B, max_len, splits).n_splits) + 512 > kNoAllocScratchBytes)
-      --splits;
-  } else if (ws_attn(D, B, max_len, plan_attn(D, B, max_len, splits).n_splits) + 512 > kNoAllocScratchBytes) {
-    return MLA_ERR_CAPACITY;
+  // The plan's unit list and partials must fit the array: an explicit split
+  // count that does not fit is refused; the automatic plan deals the tiles
+  // out to fewer CTAs until it fits.
+  const size_t cap = kNoAllocScratchBytes - 256;
+  int workers = 0;
+  if (num_splits > 0) {
+    if (ws_attn(D, B, plan_attn(D, B, max_len, num_splits)) > cap) return MLA_ERR_CAPACITY;
+  } else {
+    workers = attn_wave_workers(D);
+    while (workers > 1 && ws_attn(D, B, plan_attn(D, B, max_len, 0, workers)) > cap) workers /= 2;
+    if (ws_attn(D, B, plan_attn(D, B, max_len, 0, workers)) > cap) return MLA_ERR_CAPACITY;
   }
-  return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, scratch, kNoAllocScratchBytes, splits, o_lat,
-                      lse, as_stream(stream));
+  return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, scratch, kNoAllocScratchBytes, num_splits,
+                      o_lat, lse, as_stream(stream), workers);
 }
 
 mla_status_t mla_prefill_attn(const mla_layer_desc* D, const void* q_lat, const void* q_rope,

@@ -60,21 +60,228 @@ struct AttnCfg {
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
+#ifndef ATT_PREFETCH
+#define ATT_PREFETCH 0  // tiles of cache pages prefetched into L2 ahead of their load (0: none;
+                        // measured slower for the one-CTA kernel)
+#endif
+
 struct AttnArgs {
-  int n_h, rows, q_per_seq, span, n_splits, num_blocks, max_blocks;
+  int n_h, rows, q_per_seq, num_blocks, max_blocks;
   float scale_log2;
   const int32_t* table;
+  const uint8_t* pool;     // cache pages, 64 rows x 1152 bytes each (L2 prefetch)
   const int32_t* kv_len;   // decode: per row; nullptr for prefill
   const int32_t* q_start;  // prefill: per sequence
-  __nv_bfloat16* o_lat;    // final output (single split)
+  const int4* units;       // [segment] {row, first token, end token, partial slot or -1 (whole row)};
+                           // nullptr: CTA w does all of row w
+  const int* work;         // [CTA + 1]: first segment of each CTA (or CTA pair)
+  __nv_bfloat16* o_lat;    // final output (rows done by one unit)
   float* lse;              // final lse (may be null)
-  float* o_part;           // [split][row][head][512] partials (multi split)
-  float* lse_part;         // [split][row][head]
+  float* o_part;           // [slot][head][512] partials of rows split over several units
+  float* lse_part;         // [slot][head]
 };
 
 __device__ __forceinline__ int att_kv_len(const AttnArgs& a, int r) {
   if (a.kv_len) return a.kv_len[r];
   return a.q_start[r / a.q_per_seq] + r % a.q_per_seq + 1;
+}
+
+// Work of CTA (or CTA pair) w: segments [x, y) of the plan.  Without a plan
+// CTA w does all of row w.
+__device__ __forceinline__ int2 att_work(const AttnArgs& a, int w) {
+  if (!a.units) return make_int2(w, w + 1);
+  return make_int2(a.work[w], a.work[w + 1]);
+}
+// Segment s: {row, first token, end token, partial slot or -1}.
+__device__ __forceinline__ int4 att_seg(const AttnArgs& a, int s) {
+  if (a.units) return a.units[s];
+  return make_int4(s, 0, att_kv_len(a, s), -1);
+}
+
+// One segment as the kernels see it; n_tiles == 0 marks a segment to skip
+// (its row's kv_len is out of range: recorded as MLA_ERR_CAPACITY).
+struct SegInfo {
+  int r, t_begin, t_end, pslot, kv, n_tiles;
+};
+__device__ __forceinline__ SegInfo att_seg_info(const AttnArgs& a, int s) {
+  const int4 u = att_seg(a, s);
+  SegInfo S;
+  S.r = u.x;
+  S.t_begin = u.y;
+  S.t_end = u.z;
+  S.pslot = u.w;
+  S.kv = att_kv_len(a, S.r);
+  const bool ok = S.kv >= 1 && S.kv <= a.max_blocks * 64;
+  if (!ok) record_error(ERR_CAPACITY, 401);
+  S.n_tiles = ok && S.t_end > S.t_begin ? (S.t_end - S.t_begin + ATT_TILE - 1) / ATT_TILE : 0;
+  return S;
+}
+
+// Walks the tiles of a CTA's segments in order.  Every role of a kernel keeps
+// its own cursor; g (the tile count over all segments) indexes the pipeline's
+// barrier phases, so they run on unchanged across segment boundaries.
+struct TileCursor {
+  int s, s_end;  // current segment, end of the list
+  int j, g;      // tile within the segment, tile overall
+  int n;         // segments entered so far - 1
+  SegInfo S;
+  __device__ __forceinline__ void init(const AttnArgs& a, int2 range) {
+    s = range.x - 1;
+    s_end = range.y;
+    g = 0;
+    n = -1;
+    next_segment(a);
+  }
+  __device__ __forceinline__ void next_segment(const AttnArgs& a) {
+    j = 0;
+    while (++s < s_end) {
+      S = att_seg_info(a, s);
+      if (S.n_tiles > 0) {
+        ++n;
+        return;
+      }
+    }
+  }
+  __device__ __forceinline__ bool done() const { return s >= s_end; }
+  __device__ __forceinline__ void step(const AttnArgs& a) {
+    ++g;
+    if (++j >= S.n_tiles) next_segment(a);
+  }
+  __device__ __forceinline__ bool first() const { return j == 0; }
+  __device__ __forceinline__ bool last() const { return j == S.n_tiles - 1; }
+  __device__ __forceinline__ int tok() const { return S.t_begin + j * ATT_TILE; }
+  // the tile reaches past kv_len: rows to zero before PV
+  __device__ __forceinline__ bool zero() const { return tok() + ATT_TILE > S.kv; }
+};
+
+// Work plan (one block).  A segment is a run of 128-token tiles of one row,
+// and every CTA (or CTA pair) works through its own list of segments.
+//   automatic (splits == 0): the tiles of all rows, taken in row order, are
+//     dealt out to `workers` CTAs as equal contiguous ranges, so each CTA
+//     gets the same number of tiles (+-1) whatever the length mix; a row
+//     that straddles range boundaries becomes several segments.
+//   explicit (splits > 0): every row cut into min(splits, its tiles) equal
+//     segments, one per CTA.
+// Segments of rows cut in several get partial slots (merged by the combine
+// kernel); the others write their output directly.  Outputs:
+//   units[u]    = {row, first token, end token, slot or -1}   (row order)
+//   row_info[b] = {first segment, segments of the row, first slot, 0}
+//   work[w]     = first segment of CTA w, work[workers] = segment count
+__global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const int32_t* __restrict__ q_start,
+                                     int q_per_seq, int rows, int max_len, int workers, int splits, int max_units,
+                                     int max_slots, int4* __restrict__ units, int4* __restrict__ row_info,
+                                     int* __restrict__ work, int* __restrict__ n_units) {
+  __shared__ long long s_sum[32];
+  __shared__ int s_scan[3][1024];
+  __shared__ int s_lastw[1024];
+  __shared__ int s_per;
+  const int tid = threadIdx.x, nt = blockDim.x;
+  auto kv_of = [&](int b) -> int {
+    const int kv = kv_len ? kv_len[b] : q_start[b / q_per_seq] + b % q_per_seq + 1;
+    return min(max(kv, 0), max_len);
+  };
+  auto tiles_of = [&](int b) -> int { return (kv_of(b) + ATT_TILE - 1) / ATT_TILE; };
+  long long local = 0;
+  for (int b = tid; b < rows; b += nt) local += tiles_of(b);
+  for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+  if ((tid & 31) == 0) s_sum[tid >> 5] = local;
+  __syncthreads();
+  if (tid == 0) {
+    long long tot = 0;
+    for (int w = 0; w < nt / 32; ++w) tot += s_sum[w];
+    s_per = (int)max(1LL, (tot + workers - 1) / max(workers, 1));  // tiles per CTA (automatic)
+  }
+  __syncthreads();
+  const int per = s_per;
+  int run_tiles = 0, run_units = 0, run_slots = 0, run_lastw = -1;
+  bool bad = false;
+  for (int base = 0; base < rows; base += nt) {
+    const int b = base + tid;
+    const int tiles = b < rows ? tiles_of(b) : 0;
+    // inclusive scan of the tiles: global position of every row's first tile
+    s_scan[0][tid] = tiles;
+    __syncthreads();
+    for (int off = 1; off < nt; off <<= 1) {
+      const int a0 = tid >= off ? s_scan[0][tid - off] : 0;
+      __syncthreads();
+      s_scan[0][tid] += a0;
+      __syncthreads();
+    }
+    const int cum = run_tiles + s_scan[0][tid] - tiles;
+    int parts = 0, per_seg = 1, w0 = 0, lastw = -1;
+    if (b < rows) {
+      if (splits > 0) {
+        parts = max(1, min(splits, tiles));
+        per_seg = max(1, (tiles + parts - 1) / parts);
+        parts = max(1, (tiles + per_seg - 1) / per_seg);  // no empty segments
+      } else if (tiles > 0) {
+        w0 = cum / per;
+        lastw = (cum + tiles - 1) / per;
+        parts = lastw - w0 + 1;
+      } else {
+        w0 = lastw = min(cum / per, workers - 1);  // a row with no tiles (bad kv_len) still gets a segment
+        parts = 1;
+      }
+    }
+    s_lastw[tid] = lastw;
+    __syncthreads();
+    const int t_last = s_scan[0][nt - 1];
+    __syncthreads();
+    s_scan[1][tid] = parts;
+    s_scan[2][tid] = parts > 1 ? parts : 0;
+    __syncthreads();
+    for (int off = 1; off < nt; off <<= 1) {
+      const int a1 = tid >= off ? s_scan[1][tid - off] : 0;
+      const int a2 = tid >= off ? s_scan[2][tid - off] : 0;
+      __syncthreads();
+      s_scan[1][tid] += a1;
+      s_scan[2][tid] += a2;
+      __syncthreads();
+    }
+    const int u0 = run_units + s_scan[1][tid] - parts;
+    const int sl0 = parts > 1 ? run_slots + s_scan[2][tid] - parts : -1;
+    const bool over = b < rows && (u0 + parts > max_units || sl0 + parts > max_slots ||
+                                   (splits == 0 && lastw >= workers));
+    if (over) record_error(ERR_CAPACITY, 402);  // beyond the host's bounds: cannot happen for a valid plan
+    bad |= over;
+    if (b < rows && !over) {
+      row_info[b] = make_int4(u0, parts, sl0, 0);
+      const int kv = kv_of(b);
+      if (splits > 0) {
+        for (int q = 0; q < parts; ++q) {
+          const int t0 = min(q * per_seg * ATT_TILE, kv), t1 = min((q + 1) * per_seg * ATT_TILE, kv);
+          units[u0 + q] = make_int4(b, t0, t1, parts > 1 ? sl0 + q : -1);
+        }
+      } else {
+        // CTAs after the previous row's last one and up to this row's first
+        // start with this row's first segment
+        const int prev_w = tid > 0 ? s_lastw[tid - 1] : run_lastw;
+        for (int w = prev_w + 1; w <= w0; ++w) work[w] = u0;
+        for (int q = 0; q < parts; ++q) {
+          const int w = w0 + q;
+          if (q > 0) work[w] = u0 + q;
+          const int g0 = max(cum, w * per), g1 = min(cum + tiles, (w + 1) * per);
+          const int t0 = min((g0 - cum) * ATT_TILE, kv), t1 = min((g1 - cum) * ATT_TILE, kv);
+          units[u0 + q] = make_int4(b, t0, t1, parts > 1 ? sl0 + q : -1);
+        }
+      }
+    }
+    run_tiles += t_last;
+    run_units += s_scan[1][nt - 1];
+    run_slots += s_scan[2][nt - 1];
+    const int chunk_last = min(nt, rows - base) - 1;
+    run_lastw = s_lastw[chunk_last];
+    __syncthreads();
+  }
+  bad = __syncthreads_or(bad);
+  const int n = bad ? 0 : run_units;
+  if (splits > 0) {
+    for (int w = tid; w <= workers; w += nt) work[w] = min(w, n);
+  } else {
+    // CTAs past the last row's last one (and all of them after an error) get nothing
+    for (int w = (bad ? 0 : run_lastw + 1) + tid; w <= workers; w += nt) work[w] = n;
+  }
+  if (tid == 0) *n_units = n;
 }
 
 template <int H>
@@ -101,27 +308,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][H]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, grp = blockIdx.y, r = blockIdx.z;
-  const int kv = att_kv_len(a, r);
-  const int seq = r / a.q_per_seq;
-  const int t_begin = split * a.span;
-  const int t_end = min(t_begin + a.span, kv);
-  const int n_tiles = t_end > t_begin ? (t_end - t_begin + ATT_TILE - 1) / ATT_TILE : 0;
-  const bool direct = a.n_splits == 1;
+  // blockIdx.x = worker * (n_h / H) + head group: the head groups of one
+  // worker run side by side and share its cache tiles in L2
+  const int n_grp = a.n_h / H;
+  const int worker = blockIdx.x / n_grp, grp = blockIdx.x % n_grp;
+  const int2 range = att_work(a, worker);
   const int head0 = grp * H;
-
-  if (kv < 1 || kv > a.max_blocks * 64) {
-    if (threadIdx.x == 0) record_error(ERR_CAPACITY, 401);
-    return;
-  }
-  if (n_tiles == 0) {
-    // empty split: contributes nothing to the combine
-    if (!direct) {
-      for (int e = threadIdx.x; e < H; e += blockDim.x)
-        a.lse_part[((long long)split * a.rows + r) * a.n_h + head0 + e] = -INFINITY;
-    }
-    return;
-  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NL; ++i) {
@@ -155,34 +347,58 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     // ------------------------------------------------------------ producer
     if (elect_one()) {
       tma_prefetch_desc(&m_cache);
-      const int qrow = r * a.n_h + head0;
-      mbar_expect_tx(q_full, C::Q_BYTES);
-      for (int c = 0; c < 8; ++c) tma_load_2d(smem + C::OFF_Q + c * C::Q_CHUNK, &m_qlat, q_full, c * 64, qrow);
-      tma_load_2d(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, q_full, 0, qrow);
-      const int* trow = a.table + (long long)seq * a.max_blocks;
-      int li = 0;  // latent slot uses so far
-      for (int j = 0; j < n_tiles; ++j) {
-        const int tok = t_begin + j * ATT_TILE;
-        int blk[2];
-        for (int p = 0; p < 2; ++p) {
-          const int page = tok / 64 + p;
-          int b = a.num_blocks;  // out of range -> TMA fills zeros
-          if (page * 64 < kv) {
-            b = trow[page];
-            if (b < 0 || b >= a.num_blocks) {
-              record_error(ERR_CAPACITY, 402);
-              b = a.num_blocks;
-            }
+      // cache block of page `page` of the cursor's row; past the row:
+      // num_blocks (out of range: TMA reads zeros)
+      auto page_block = [&](const TileCursor& c, int page) -> int {
+        int b = a.num_blocks;
+        if (page * 64 < c.S.kv) {
+          b = a.table[(long long)(c.S.r / a.q_per_seq) * a.max_blocks + page];
+          if (b < 0 || b >= a.num_blocks) {
+            record_error(ERR_CAPACITY, 402);
+            b = a.num_blocks;
           }
-          blk[p] = b;
         }
-        const int rs = j % C::NR;
-        if (j >= C::NR && !mbar_wait(&rope_empty[rs], ((j / C::NR) - 1) & 1, abort_flag, 404)) break;
+        return b;
+      };
+      // Pages are prefetched into L2 ATT_PREFETCH tiles ahead of their TMA
+      // loads, which then see L2 rather than HBM latency.
+      constexpr uint32_t PAGE_BYTES = 64u * (ATT_DC + ATT_DR) * 2u;
+      TileCursor c, cf;
+      c.init(a, range);
+      cf = c;
+      auto prefetch = [&]() {
+        if (ATT_PREFETCH > 0 && !cf.done()) {
+          for (int p = 0; p < 2; ++p) {
+            const int b = page_block(cf, cf.tok() / 64 + p);
+            if (b < a.num_blocks) prefetch_l2_bulk(a.pool + (size_t)b * PAGE_BYTES, PAGE_BYTES);
+          }
+          cf.step(a);
+        }
+      };
+      if (!cf.done()) cf.step(a);
+      for (int i = 0; i < ATT_PREFETCH; ++i) prefetch();
+      bool ok = true;
+      while (ok && !c.done()) {
+        const int g = c.g;
+        if (c.first()) {
+          // the queries of the segment's row; the buffer is free once the
+          // previous segment's last QK is done
+          if (g >= 1 && !mbar_wait(&s_full[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, 405)) break;
+          const int qrow = c.S.r * a.n_h + head0;
+          mbar_expect_tx(q_full, C::Q_BYTES);
+          for (int k = 0; k < 8; ++k) tma_load_2d(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, q_full, k * 64, qrow);
+          tma_load_2d(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, q_full, 0, qrow);
+        }
+        prefetch();
+        int blk[2];
+        for (int p = 0; p < 2; ++p) blk[p] = page_block(c, c.tok() / 64 + p);
+        const int rs = g % C::NR;
+        if (g >= C::NR && !mbar_wait(&rope_empty[rs], ((g / C::NR) - 1) & 1, abort_flag, 404)) break;
         uint8_t* rdst = smem + C::OFF_ROPE + rs * C::ROPE_SLOT;
         mbar_expect_tx(&rope_full[rs], C::ROPE_SLOT);
         for (int p = 0; p < 2; ++p) tma_load_3d(rdst + p * 8192, &m_cache, &rope_full[rs], ATT_DC, 0, blk[p]);
-        bool ok = true;
-        for (int m = 0; m < 4 && ok; ++m, ++li) {
+        for (int m = 0; m < 4; ++m) {
+          const int li = 4 * g + m;  // latent slot uses so far
           const int s = li % C::NL;
           if (li >= C::NL && !mbar_wait(&lat_empty[s], ((li / C::NL) - 1) & 1, abort_flag, 403)) {
             ok = false;
@@ -194,7 +410,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             for (int p = 0; p < 2; ++p)
               tma_load_3d(dst + hh * 16384 + p * 8192, &m_cache, &lat_full[s], m * 128 + hh * 64, 0, blk[p]);
         }
-        if (!ok) break;
+        c.step(a);
       }
     }
   } else if (warp == 1) {
@@ -210,15 +426,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const uint32_t lat_base = smem_u32(smem + C::OFF_LAT);
       const uint32_t rope_base = smem_u32(smem + C::OFF_ROPE);
       const uint32_t p_base = smem_u32(smem + C::OFF_P);
-      bool ok = mbar_wait(q_full, 0, abort_flag, 411);
-      int jq = 0, cq = 0;    // next QK tile and chunk
-      bool sbuf_ok = false;  // S buffer of tile jq released by the softmax
-      int jp = 0;            // next PV tile
+      TileCursor cq, cp;  // next QK tile, next PV tile
+      cq.init(a, range);
+      cp = cq;
+      int kq = 0;            // next QK chunk of tile cq
+      bool sbuf_ok = false;  // S buffer of tile cq released by the softmax
+      int q_seen = -1;       // segment whose queries have landed
+      bool ok = true;
       uint64_t t_idle = 0;
       uint32_t spins = 0;
-      while (ok && jp < n_tiles) {
+      while (ok && !cp.done()) {
         bool prog = false;
-        if (jp < jq && mbar_test(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1)) {
+        const int jp = cp.g;
+        if (jp < cq.g && mbar_test(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1)) {
           tc_fence_after();
           const int pb = jp & 1;
           for (int m = 0; m < 4; ++m) {
@@ -229,28 +449,30 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
               const uint64_t ad = smem_desc(va + kk * 2048, 16384, 1024, SW128);
               const uint64_t bd = smem_desc(p_base + pb * C::P_BYTES + kk * 16 * 2 * H, C::P_BYTES, 8 * 2 * H,
                                             C::P_LAYOUT);
-              mma_bf16_ss(tO + m * H, ad, bd, id_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+              mma_bf16_ss(tO + m * H, ad, bd, id_pv, (cp.j > 0 || kk > 0) ? 1u : 0u);
             }
             mma_commit(&lat_empty[s]);
           }
           mma_commit(&pv_done[pb]);
-          ++jp;
+          cp.step(a);
           prog = true;
         }
-        if (jq < n_tiles) {
+        if (!cq.done()) {
+          const int jq = cq.g;
           const int sb = jq & 1;
           if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_test(smem_u32(&s_free[sb]), ((jq >> 1) - 1) & 1);
-          if (sbuf_ok) {
+          if (q_seen != cq.n && mbar_test(smem_u32(q_full), cq.n & 1)) q_seen = cq.n;
+          if (sbuf_ok && q_seen == cq.n) {
             bool ready;
             uint32_t ka;
             int qchunk;  // chunk of Q: 0..7 latent, 8 rope
-            if (cq == 0) {
+            if (kq == 0) {
               const int rs = jq % C::NR;
               ready = mbar_test(smem_u32(&rope_full[rs]), (jq / C::NR) & 1);
               ka = rope_base + rs * C::ROPE_SLOT;
               qchunk = 8;
             } else {
-              const int c = cq - 1;
+              const int c = kq - 1;
               const int li = jq * 4 + c / 2;
               const int s = li % C::NL;
               ready = (c & 1) || mbar_test(smem_u32(&lat_full[s]), (li / C::NL) & 1);
@@ -263,13 +485,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ad = smem_desc(ka + kk * 32, 16, 1024, SW128);
                 const uint64_t bd = smem_desc(q_base + qchunk * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
-                mma_bf16_ss(tS + sb * H, ad, bd, id_qk, (cq | kk) != 0 ? 1u : 0u);
+                mma_bf16_ss(tS + sb * H, ad, bd, id_qk, (kq | kk) != 0 ? 1u : 0u);
               }
-              if (cq == 0) mma_commit(&rope_empty[jq % C::NR]);
-              if (++cq == 9) {
+              if (kq == 0) mma_commit(&rope_empty[jq % C::NR]);
+              if (++kq == 9) {
                 mma_commit(&s_full[sb]);
-                ++jq;
-                cq = 0;
+                cq.step(a);
+                kq = 0;
                 sbuf_ok = false;
               }
               prog = true;
@@ -289,7 +511,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           } else if (now - t_idle > g_spin_limit_ns) {
             record_error(ERR_TIMEOUT, 412);
             *abort_flag = 1;
-            break;
+            ok = false;
           }
         }
       }
@@ -301,11 +523,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int tr = q * 32 + lane;           // token row within a tile (TMEM lane)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     float m_run[H], l_part[H];
-#pragma unroll
-    for (int h = 0; h < H; ++h) {
-      m_run[h] = -INFINITY;
-      l_part[h] = 0.f;
-    }
     uint8_t* p_smem = smem + C::OFF_P;
     uint32_t gphase = 0;
     // bounded 128-thread barrier (a bar.sync could wait forever on a warp
@@ -317,8 +534,18 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       return r;
     };
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
+    TileCursor c;
+    c.init(a, range);
+    while (ok && !c.done()) {
+      const int j = c.g;
       const int sb = j & 1;
+      if (c.first()) {
+#pragma unroll
+        for (int h = 0; h < H; ++h) {
+          m_run[h] = -INFINITY;
+          l_part[h] = 0.f;
+        }
+      }
       if (!mbar_wait(&s_full[sb], (j >> 1) & 1, abort_flag, 421)) {
         ok = false;
         break;
@@ -329,8 +556,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_free[sb]);
-      const int tok = t_begin + j * ATT_TILE + tr;
-      const bool valid = tok < t_end;
+      const int tok = c.tok() + tr;
+      const bool valid = tok < c.S.t_end;
       // tile max per head: warp redux, then exchange across the 4 warps
       float* rb = red + (j & 1) * 4 * H;
 #pragma unroll
@@ -351,7 +578,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         m_new[h] = fmaxf(m_run[h], tm);
         grow |= (m_new[h] > m_run[h] + ATT_RESCALE_LOG2);
       }
-      if (j == 0) {
+      if (c.first()) {
+        // PV of a segment's first tile overwrites O^T
 #pragma unroll
         for (int h = 0; h < H; ++h) m_run[h] = m_new[h];
       } else if (grow) {
@@ -396,13 +624,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       uint8_t* prow = p_smem + sb * C::P_BYTES;
 #pragma unroll
-      for (int c = 0; c < H / 8; ++c) {
-        const uint32_t off = swizzle_off((uint32_t)(tr * 2 * H + c * 16), C::P_LAYOUT);
-        *reinterpret_cast<uint4*>(prow + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      for (int cc = 0; cc < H / 8; ++cc) {
+        const uint32_t off = swizzle_off((uint32_t)(tr * 2 * H + cc * 16), C::P_LAYOUT);
+        *reinterpret_cast<uint4*>(prow + off) =
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
       }
-      if (j == n_tiles - 1 && t_begin + j * ATT_TILE + ATT_TILE > kv) {
-        // last tile: zero the latent rows past kv_len before PV reads them
-        const int first = kv - (t_begin + j * ATT_TILE);
+      if (c.zero()) {
+        // the row's last tile: zero the latent rows past kv_len before PV reads them
+        const int first = c.S.kv - c.tok();
         for (int m = 0; m < 4; ++m) {
           uint8_t* slot = smem + C::OFF_LAT + ((j * 4 + m) % C::NL) * C::LAT_SLOT;
           for (int e = first * 8 + tr; e < ATT_TILE * 8; e += 128) {
@@ -417,57 +646,64 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[sb]);
-    }
-    // ------------------------------------------------------------ epilogue
-    // l per head: sum of the per-thread partials over the 128 token rows
-    ok = ok && group_sync(426);
-    float* lred = red;  // reuse [4][H]
+      if (c.last()) {
+        // ---------------------------------------------------------- epilogue of the segment
+        // O^T is read out before this thread writes the next segment's first
+        // P, which is what PV of that tile (overwriting O^T) waits for.
+        const SegInfo& S = c.S;
+        const bool direct = S.pslot < 0;
+        // l per head: sum of the per-thread partials over the 128 token rows
+        ok = ok && group_sync(426);
+        float* lred = red;  // reuse [4][H]
 #pragma unroll
-    for (int h = 0; h < H; ++h) {
-      const float ws = warp_sum(l_part[h]);
-      if (ok && lane == (h & 31)) lred[sw * H + h] = ws;
-    }
-    ok = group_sync(427) && ok;
-    float l_tot[H];
+        for (int h = 0; h < H; ++h) {
+          const float ws = warp_sum(l_part[h]);
+          if (ok && lane == (h & 31)) lred[sw * H + h] = ws;
+        }
+        ok = group_sync(427) && ok;
+        float l_tot[H];
 #pragma unroll
-    for (int h = 0; h < H; ++h) l_tot[h] = lred[h] + lred[H + h] + lred[2 * H + h] + lred[3 * H + h];
-    const int last = n_tiles - 1;
-    ok = ok && mbar_wait(&pv_done[last & 1], (last >> 1) & 1, abort_flag, 424);
-    tc_fence_after();
-    // thread = latent row d = 128*m + tr of O^T, registers = heads
+        for (int h = 0; h < H; ++h) l_tot[h] = lred[h] + lred[H + h] + lred[2 * H + h] + lred[3 * H + h];
+        ok = ok && mbar_wait(&pv_done[j & 1], (j >> 1) & 1, abort_flag, 424);
+        tc_fence_after();
+        // thread = latent row d = 128*m + tr of O^T, registers = heads
 #pragma unroll 1
-    for (int m = 0; m < 4; ++m) {
-      float o[H];
-      tmem_ld32<H>(tO + m * H + lane_off, o);
-      tmem_wait_ld();
-      if (!ok) continue;
-      const int d = m * 128 + tr;
+        for (int m = 0; m < 4; ++m) {
+          float o[H];
+          tmem_ld32<H>(tO + m * H + lane_off, o);
+          tmem_wait_ld();
+          if (!ok) continue;
+          const int d = m * 128 + tr;
 #pragma unroll
-      for (int h = 0; h < H; ++h) {
-        const float val = o[h] / l_tot[h];
-        const long long oi = ((long long)r * a.n_h + head0 + h) * ATT_DC + d;
-        if (direct) {
-          a.o_lat[oi] = __float2bfloat16_rn(val);
-        } else {
-          a.o_part[(long long)split * a.rows * a.n_h * ATT_DC + oi] = val;
+          for (int h = 0; h < H; ++h) {
+            const float val = o[h] / l_tot[h];
+            if (direct) {
+              a.o_lat[((long long)S.r * a.n_h + head0 + h) * ATT_DC + d] = __float2bfloat16_rn(val);
+            } else {
+              a.o_part[((long long)S.pslot * a.n_h + head0 + h) * ATT_DC + d] = val;
+            }
+          }
         }
-      }
-    }
-    if (ok && sw == 0 && lane < H) {
-      float mm = 0.f, ll = 0.f;
+        tc_fence_before();
+        if (ok && sw == 0 && lane < H) {
+          float mm = 0.f, ll = 0.f;
 #pragma unroll
-      for (int h = 0; h < H; ++h)
-        if (h == lane) {
-          mm = m_run[h];
-          ll = l_tot[h];
+          for (int h = 0; h < H; ++h)
+            if (h == lane) {
+              mm = m_run[h];
+              ll = l_tot[h];
+            }
+          const float lse = (mm + log2f(ll)) * 0.69314718055994531f;
+          if (direct) {
+            if (a.lse) a.lse[(long long)S.r * a.n_h + head0 + lane] = lse;
+          } else {
+            a.lse_part[(long long)S.pslot * a.n_h + head0 + lane] = lse;
+          }
         }
-      const float lse = (mm + log2f(ll)) * 0.69314718055994531f;
-      const long long li = (long long)r * a.n_h + head0 + lane;
-      if (direct) {
-        if (a.lse) a.lse[li] = lse;
-      } else {
-        a.lse_part[(long long)split * a.rows * a.n_h + li] = lse;
+        // the 4 x H sums are read by every thread before the red buffer is reused
+        ok = group_sync(428) && ok;
       }
+      c.step(a);
     }
   }
   tc_fence_before();
@@ -475,37 +711,35 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-// Merge split partials: lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
-__global__ void mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, int n_splits,
-                                   int rows, int n_h, __nv_bfloat16* __restrict__ o_lat, float* __restrict__ lse) {
-  const int rh = blockIdx.x;  // row * n_h + head
-  const long long stride_o = (long long)rows * n_h * ATT_DC;
-  const long long stride_l = (long long)rows * n_h;
+// Merge the partials of rows cut into several units:
+// lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
+__global__ void mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                                   const int4* __restrict__ row_info, int n_h, __nv_bfloat16* __restrict__ o_lat,
+                                   float* __restrict__ lse) {
+  const int r = blockIdx.x / n_h, h = blockIdx.x % n_h;
+  const int4 info = row_info[r];
+  const int n_parts = info.y, slot0 = info.z;
+  if (n_parts <= 1) return;  // written directly by its unit
   float mx = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) mx = fmaxf(mx, lse_part[s * stride_l + rh]);
+  for (int s = 0; s < n_parts; ++s) mx = fmaxf(mx, lse_part[(long long)(slot0 + s) * n_h + h]);
   float tot = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const float v = lse_part[s * stride_l + rh];
-    tot += v == -INFINITY ? 0.f : expf(v - mx);
-  }
+  for (int s = 0; s < n_parts; ++s) tot += expf(lse_part[(long long)(slot0 + s) * n_h + h] - mx);
   const float lse_all = mx + logf(tot);
   for (int d = threadIdx.x * 4; d < ATT_DC; d += blockDim.x * 4) {
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_splits; ++s) {
-      const float v = lse_part[s * stride_l + rh];
-      if (v == -INFINITY) continue;
-      const float wgt = expf(v - lse_all);
-      const float4 x = *reinterpret_cast<const float4*>(o_part + s * stride_o + (long long)rh * ATT_DC + d);
+    for (int s = 0; s < n_parts; ++s) {
+      const float wgt = expf(lse_part[(long long)(slot0 + s) * n_h + h] - lse_all);
+      const float4 x = *reinterpret_cast<const float4*>(o_part + ((long long)(slot0 + s) * n_h + h) * ATT_DC + d);
       acc.x += wgt * x.x;
       acc.y += wgt * x.y;
       acc.z += wgt * x.z;
       acc.w += wgt * x.w;
     }
-    __nv_bfloat16* dst = o_lat + (long long)rh * ATT_DC + d;
+    __nv_bfloat16* dst = o_lat + ((long long)r * n_h + h) * ATT_DC + d;
     *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc.x, acc.y);
     *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc.z, acc.w);
   }
-  if (lse && threadIdx.x == 0) lse[rh] = lse_all;
+  if (lse && threadIdx.x == 0) lse[(long long)r * n_h + h] = lse_all;
 }
 
 }  // namespace mla

@@ -43,6 +43,10 @@
 
 namespace mla {
 
+#ifndef PAIR_PREFETCH
+#define PAIR_PREFETCH 1  // tiles of own pages prefetched into L2 ahead of their load
+#endif
+
 struct PairCfg {
   static constexpr int THREADS = 224;
   static constexpr int Q_CHUNK = 64 * 128;        // 64 heads x 64 columns
@@ -97,28 +101,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int split = blockIdx.x >> 1, r = blockIdx.z;
-  const int kv = att_kv_len(a, r);
-  const int seq = r / a.q_per_seq;
-  const int t_begin = split * a.span;
-  const int t_end = min(t_begin + a.span, kv);
-  const int n_tiles = t_end > t_begin ? (t_end - t_begin + ATT_TILE - 1) / ATT_TILE : 0;
-  const bool direct = a.n_splits == 1;
+  // both CTAs of the pair walk the same segment list
+  const int worker = blockIdx.x >> 1;
+  const int2 range = att_work(a, worker);
   const int head0 = (int)rank * 64;
-  const int tunit = rank == 0 ? r * a.n_splits + split : -1;  // trace slot (leader only)
+  const int tunit = rank == 0 ? worker : -1;  // trace slot (leader only)
   (void)tunit;
-
-  // both CTAs of the pair take the same early exits (same row and split)
-  if (kv < 1 || kv > a.max_blocks * 64) {
-    if (threadIdx.x == 0) record_error(ERR_CAPACITY, 501);
-    return;
-  }
-  if (n_tiles == 0) {
-    if (!direct)
-      for (int e = threadIdx.x; e < 64; e += blockDim.x)
-        a.lse_part[((long long)split * a.rows + r) * a.n_h + head0 + e] = -INFINITY;
-    return;
-  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NP; ++i) {
@@ -149,14 +137,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 0, 0);
   const uint32_t tS = tmem;         // S buffers: columns [0,64) and [64,128)
   const uint32_t tO = tmem + 128;   // O: columns [128,256) (d_c 0..255) and [256,384) (256..511)
-  const int* trow = a.table + (long long)seq * a.max_blocks;
 
-  // the last tile of a unit that reaches past kv_len: rows to zero before PV
-  auto needs_zero = [&](int j) -> bool { return t_begin + j * ATT_TILE + ATT_TILE > kv; };
-  auto page_block = [&](int page) -> int {
-    int b = a.num_blocks;  // past the sequence: TMA reads zeros
-    if (page * 64 < kv) {
-      b = trow[page];
+  // cache block of page `page` of the cursor's row; past the row: num_blocks
+  // (out of range: TMA reads zeros)
+  auto page_block = [&](const TileCursor& c, int page) -> int {
+    int b = a.num_blocks;
+    if (page * 64 < c.S.kv) {
+      b = a.table[(long long)(c.S.r / a.q_per_seq) * a.max_blocks + page];
       if (b < 0 || b >= a.num_blocks) {
         record_error(ERR_CAPACITY, 502);
         b = a.num_blocks;
@@ -164,9 +151,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     }
     return b;
   };
-  // pair slot of latent pair k of tile j, and how often that slot was used before
-  auto slot_of = [](int j, int k) -> int { return (4 * j + k) % C::NP; };
-  auto use_of = [](int j, int k) -> int { return (4 * j + k) / C::NP; };
+  // pair slot of latent pair k of tile g, and how often that slot was used before
+  auto slot_of = [](int g, int k) -> int { return (4 * g + k) % C::NP; };
+  auto use_of = [](int g, int k) -> int { return (4 * g + k) / C::NP; };
   // Pair k of a tile serves PV instruction k >> 1 over the tokens of page k & 1.
   // The CTA whose own page is k & 1 keeps its own columns there; the other CTA
   // refills the slot with columns 2*(2*(k>>1) + rank) .. +1 of page k & 1.
@@ -175,47 +162,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     // ------------------------------------------------------------ own-page producer
     // Per tile two TMA instructions: the RoPE chunk (8 KB) and all eight
     // latent chunks of the own page (64 KB, landing in the tile's four
-    // consecutive pair slots).  Few large boxes keep one issuing thread at
-    // full HBM rate.
+    // consecutive pair slots); per segment the queries of its row.
     if (elect_one()) {
       tma_prefetch_desc(&m_page8);
-      if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
       const uint32_t lq = mapa_shared(smem_u32(q_full), 0);
-      const int qrow = r * a.n_h + head0;
-      for (int c = 0; c < 8; ++c) tma_load_2d_pair(smem + C::OFF_Q + c * C::Q_CHUNK, &m_qlat, lq, c * 64, qrow);
-      tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
-      const int first_page = t_begin / 64 + (int)rank;
       const uint32_t l_rope = mapa_shared(smem_u32(rope_full), 0);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int blk = page_block(first_page + 2 * j);
-        // the RoPE slot is free once QK(j-1) is done
-        if (j >= 1 && !mbar_wait(&s_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 503)) break;
+      // Own pages are prefetched into L2 PAIR_PREFETCH tiles ahead: the TMA
+      // loads below, and the other CTA's refills from this page, then see L2
+      // rather than HBM latency, which no shared-memory ring could cover.
+      constexpr uint32_t PAGE_BYTES = 64u * (ATT_DC + ATT_DR) * 2u;
+      TileCursor c, cf;
+      c.init(a, range);
+      cf = c;
+      auto prefetch = [&]() {
+        if (!cf.done()) {
+          const int page = cf.tok() / 64 + (int)rank;
+          const int b = page_block(cf, page);
+          if (b < a.num_blocks) prefetch_l2_bulk(a.pool + (size_t)b * PAGE_BYTES, PAGE_BYTES);
+          cf.step(a);
+        }
+      };
+      if (!cf.done()) cf.step(a);
+      for (int i = 0; i < PAIR_PREFETCH; ++i) prefetch();
+      while (!c.done()) {
+        const int g = c.g;
+        // the RoPE slot, and at a segment's start the Q buffer, are free once
+        // QK(g-1) is done
+        if (g >= 1 && !mbar_wait(&s_full[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, 503)) break;
+        if (c.first()) {
+          if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
+          const int qrow = c.S.r * a.n_h + head0;
+          for (int k = 0; k < 8; ++k)
+            tma_load_2d_pair(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, lq, k * 64, qrow);
+          tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
+        }
+        prefetch();
+        const int blk = page_block(c, c.tok() / 64 + (int)rank);
         if (rank == 0) mbar_expect_tx(rope_full, 2 * C::ROPE);
         tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, 8, blk);
-        MLA_TRACE_EVENT(tunit, 1, j);
-        // the tile's four pair slots were last used by PV(j-2)
-        if (j >= 2 && !mbar_wait(&pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, 504)) break;
-        uint64_t* of = &own_full[j & 1];
+        MLA_TRACE_EVENT(tunit, 1, g);
+        // the tile's four pair slots were last used by PV(g-2)
+        if (g >= 2 && !mbar_wait(&pv_done[g & 1], ((g - 2) >> 1) & 1, abort_flag, 504)) break;
+        uint64_t* of = &own_full[g & 1];
         if (rank == 0) mbar_expect_tx(of, 2 * 4 * C::PAIR);
-        tma_load_4d_pair(smem + C::OFF_PAIR + slot_of(j, 0) * C::PAIR, &m_page8, mapa_shared(smem_u32(of), 0), 0, 0,
+        tma_load_4d_pair(smem + C::OFF_PAIR + slot_of(g, 0) * C::PAIR, &m_page8, mapa_shared(smem_u32(of), 0), 0, 0,
                          0, blk);
-        MLA_TRACE_EVENT(tunit, 2, j);
+        MLA_TRACE_EVENT(tunit, 2, g);
+        c.step(a);
       }
     }
   } else if (warp == 6) {
     // ------------------------------------------------------------ other-page producer
-    for (int j = 0; j < n_tiles; ++j) {
-      const int tok = t_begin + j * ATT_TILE;
-      const bool zero = needs_zero(j);
-      bool ok = true;
+    TileCursor c;
+    c.init(a, range);
+    int nz = 0;  // zero tiles so far (phase of z_land)
+    bool ok = true;
+    while (ok && !c.done()) {
+      const int g = c.g;
+      const bool zero = c.zero();
       if (lane == 0) {
         int zk = 0;  // refills of this tile that land on z_land
         for (int k = 0; k < 4 && ok; ++k) {
-          const int s = slot_of(j, k), u = use_of(j, k);
+          const int s = slot_of(g, k), u = use_of(g, k);
           if ((k & 1) == (int)rank) continue;  // kept by this CTA
-          ok = mbar_wait(&qk_done[s], u & 1, abort_flag, 505);  // QK(j) has read this pair
+          ok = mbar_wait(&qk_done[s], u & 1, abort_flag, 505);  // QK(g) has read this pair
           if (!ok) break;
-          const int b = page_block(tok / 64 + (k & 1));
+          const int b = page_block(c, c.tok() / 64 + (k & 1));
           const int c0 = 2 * (2 * (k >> 1) + (int)rank);  // columns this CTA multiplies in instruction k >> 1
           uint8_t* dst = smem + C::OFF_PAIR + s * C::PAIR;
           if (!zero) {
@@ -233,14 +245,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       if (zero) {
         // every pair this CTA presents to PV — refilled ones once landed, kept
         // ones once QK is done with them — gets its rows past kv_len zeroed
-        const int first = kv - tok;
+        const int first = c.S.kv - c.tok();
         int zi = 0;
         for (int k = 0; k < 4 && ok; ++k) {
-          const int s = slot_of(j, k);
+          const int s = slot_of(g, k);
           const bool refilled = (k & 1) != (int)rank;
           if (lane == 0)
-            ok = refilled ? mbar_wait(&z_land[zi], 0, abort_flag, 506)
-                          : mbar_wait(&qk_done[s], use_of(j, k) & 1, abort_flag, 507);
+            ok = refilled ? mbar_wait(&z_land[zi], nz & 1, abort_flag, 506)
+                          : mbar_wait(&qk_done[s], use_of(g, k) & 1, abort_flag, 507);
           if (refilled) ++zi;
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
@@ -255,8 +267,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive_cluster(mapa_shared(smem_u32(last_ready), 0));
-        if (!ok) break;
+        ++nz;
       }
+      c.step(a);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
@@ -267,32 +280,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       const uint32_t rope_base = smem_u32(smem + C::OFF_ROPE);
       const uint32_t pair0 = smem_u32(smem + C::OFF_PAIR);
       const uint32_t p_base = smem_u32(smem + C::OFF_P);
+      TileCursor cq, cp, cpost;  // next QK tile, next PV tile, PV tile + 2
+      cq.init(a, range);
+      cp = cq;
+      cpost = cq;
       // Byte counts of the refills the peer performs (pairs k = 0, 2) are
       // posted here, each as soon as the slot's previous refill has been
       // consumed by PV; the leader's own refills post theirs themselves.
-      auto post_peer_refills = [&](int j) {
-        if (j < n_tiles && !needs_zero(j))
-          for (int k = 0; k < 4; k += 2) mbar_expect_tx(&oth_full[slot_of(j, k)], C::PAIR);
+      auto post_peer_refill = [&](int k) {
+        if (!cpost.done() && !cpost.zero()) mbar_expect_tx(&oth_full[slot_of(cpost.g, k)], C::PAIR);
       };
-      post_peer_refills(0);
-      post_peer_refills(1);
-      bool ok = mbar_wait(q_full, 0, abort_flag, 511);
+      for (int t = 0; t < 2; ++t) {
+        post_peer_refill(0);
+        post_peer_refill(2);
+        if (!cpost.done()) cpost.step(a);
+      }
       // Work is issued in batches (a tile's 32 latent QK MMAs at once, PV pair
       // by pair): every barrier probe between MMAs costs issue slots.
-      int jq = 0, jp = 0, pv_k = 0;  // next QK tile, next PV tile, next pair of PV(jp)
-      bool sbuf_ok = false, rope_pending = false, p_ok = false;
+      int pv_k = 0;  // next pair of PV(cp)
+      int q_seen = -1;  // segment whose queries have landed
+      int nz = 0;       // zero tiles passed by PV (phase of last_ready)
+      bool sbuf_ok = false, rope_pending = false, p_ok = false, ok = true;
       uint64_t t_idle = 0;
       uint32_t spins = 0;
-      while (ok && jp < n_tiles) {
+      while (ok && !cp.done()) {
         bool prog = false;
-        // PV(jp) first: it frees the slots that later tiles' loads wait for
-        if (jp < jq) {
+        // PV first: it frees the slots that later tiles' loads wait for
+        if (cp.g < cq.g) {
+          const int jp = cp.g;
           if (!p_ok) p_ok = mbar_test_cluster(smem_u32(p_full), jp & 1);
           if (p_ok) {
-            const bool zero = needs_zero(jp);
+            const bool zero = cp.zero();
             while (pv_k < 4) {
               const int s = slot_of(jp, pv_k), u = use_of(jp, pv_k);
-              const bool ready = zero ? mbar_test_cluster(smem_u32(last_ready), 0)
+              const bool ready = zero ? mbar_test_cluster(smem_u32(last_ready), nz & 1)
                                       : mbar_test(smem_u32(&oth_full[s]), u & 1);
               if (!ready) break;
               if (pv_k == 0) MLA_TRACE_EVENT(tunit, 14, jp);
@@ -303,39 +324,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ad = smem_desc(p_base + p * 8192 + kk * 32, 16, 1024, SW128);
                 const uint64_t bd = smem_desc(pb + kk * 2048, 8192, 1024, SW128);
-                mma_bf16_pair(tO + 128 * i, ad, bd, id_pv, (jp > 0 || p > 0 || kk > 0) ? 1u : 0u);
+                mma_bf16_pair(tO + 128 * i, ad, bd, id_pv, (cp.j > 0 || p > 0 || kk > 0) ? 1u : 0u);
               }
-              if ((pv_k & 1) == 0 && jp + 2 < n_tiles && !needs_zero(jp + 2))
-                mbar_expect_tx(&oth_full[slot_of(jp + 2, pv_k)], C::PAIR);
+              // a zero tile's slots had no refill on oth_full: close that phase
+              if (zero) mbar_arrive(&oth_full[s]);
+              if ((pv_k & 1) == 0) post_peer_refill(pv_k);
               ++pv_k;
               prog = true;
             }
             if (pv_k == 4) {
               MLA_TRACE_EVENT(tunit, 5, jp);
               mma_commit_pair(&pv_done[jp & 1]);
-              ++jp;
+              if (zero) ++nz;
+              cp.step(a);
+              if (!cpost.done()) cpost.step(a);
               pv_k = 0;
               p_ok = false;
             }
           }
         }
-        if (jq < n_tiles) {
+        if (!cq.done()) {
+          const int jq = cq.g;
           if (!rope_pending) {
             if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_test_cluster(smem_u32(&s_free[jq & 1]), ((jq >> 1) - 1) & 1);
-            if (sbuf_ok && mbar_test(smem_u32(&own_full[jq & 1]), (jq >> 1) & 1)) {
+            if (q_seen != cq.n && mbar_test(smem_u32(q_full), cq.n & 1)) q_seen = cq.n;
+            if (sbuf_ok && q_seen == cq.n && mbar_test(smem_u32(&own_full[jq & 1]), (jq >> 1) & 1)) {
               MLA_TRACE_EVENT(tunit, 6, jq);
               tc_fence_after();
               // the 8 latent chunks, pair by pair; each pair's commit lets the
               // other CTA refill that slot
-              for (int c = 0; c < 8; ++c) {
-                const uint32_t kb = pair0 + slot_of(jq, c >> 1) * C::PAIR + (c & 1) * 8192;
+              for (int k = 0; k < 8; ++k) {
+                const uint32_t kb = pair0 + slot_of(jq, k >> 1) * C::PAIR + (k & 1) * 8192;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                  const uint64_t ad = smem_desc(q_base + c * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
+                  const uint64_t ad = smem_desc(q_base + k * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
                   const uint64_t bd = smem_desc(kb + kk * 32, 16, 1024, SW128);
-                  mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qk, (c | kk) != 0 ? 1u : 0u);
+                  mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qk, (k | kk) != 0 ? 1u : 0u);
                 }
-                if (c & 1) mma_commit_pair(&qk_done[slot_of(jq, c >> 1)]);
+                if (k & 1) mma_commit_pair(&qk_done[slot_of(jq, k >> 1)]);
               }
               rope_pending = true;
               prog = true;
@@ -351,7 +377,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             }
             MLA_TRACE_EVENT(tunit, 7, jq);
             mma_commit_pair(&s_full[jq & 1]);
-            ++jq;
+            cq.step(a);
             rope_pending = false;
             sbuf_ok = false;
             prog = true;
@@ -370,7 +396,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           } else if (now - t_idle > g_spin_limit_ns) {
             record_error(ERR_TIMEOUT, 512);
             *abort_flag = 1;
-            break;
+            ok = false;
           }
         }
       }
@@ -393,7 +419,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     };
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles && ok; ++j) {
+    TileCursor c;
+    c.init(a, range);
+    while (ok && !c.done()) {
+      const int j = c.g;
+      if (c.first()) {
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
       if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, 521)) {
         ok = false;
         break;
@@ -402,16 +435,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       tc_fence_after();
       float s[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32<16>(tS + (j & 1) * 64 + c * 16 + lane_off, s + 16 * c);
+      for (int cc = 0; cc < 4; ++cc) tmem_ld32<16>(tS + (j & 1) * 64 + cc * 16 + lane_off, s + 16 * cc);
       tmem_wait_ld();
       tc_fence_before();
-      const int tok0 = t_begin + j * ATT_TILE + 64 * g;
-      const int nvalid = min(64, max(0, t_end - tok0));
+      const int tok0 = c.tok() + 64 * g;
+      const int nvalid = min(64, max(0, c.S.t_end - tok0));
       float pmax = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        s[c] = c < nvalid ? s[c] * a.scale_log2 : -INFINITY;
-        pmax = fmaxf(pmax, s[c]);
+      for (int cc = 0; cc < 64; ++cc) {
+        s[cc] = cc < nvalid ? s[cc] * a.scale_log2 : -INFINITY;
+        pmax = fmaxf(pmax, s[cc]);
       }
       float* rb = red + (j & 1) * 128;
       rb[L] = pmax;
@@ -437,20 +470,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         tc_fence_after();
       }
       const bool grow = __any_sync(0xffffffffu, m_new > m_run + ATT_RESCALE_LOG2);
-      if (j == 0) {
-        m_run = m_new;
+      if (c.first()) {
+        m_run = m_new;  // PV of a segment's first tile overwrites O
       } else if (grow) {
         const float alpha = exp2_approx(m_run - m_new);
         l_run *= alpha;
         m_run = m_new;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 16) {
+        for (int cc = 0; cc < 256; cc += 16) {
           float o[16];
-          tmem_ld32<16>(tO + c + lane_off, o);
+          tmem_ld32<16>(tO + cc + lane_off, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) o[e] *= alpha;
-          tmem_st32<16>(tO + c + lane_off, o);
+          tmem_st32<16>(tO + cc + lane_off, o);
         }
         tmem_wait_st();
       }
@@ -480,48 +513,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           mbar_arrive_cluster(l_pfull);
         MLA_TRACE_EVENT(tunit, 10, j);
       }
-    }
-    // ------------------------------------------------------------ epilogue
-    float* lred = red + 256;
-    lred[L] = l_run;
-    ok = group_sync(524) && ok;
-    const float l_tot = l_run + lred[L ^ 64];
-    const int last = n_tiles - 1;
-    ok = ok && mbar_wait(&pv_done[last & 1], (last >> 1) & 1, abort_flag, 525);
-    tc_fence_after();
-    const float inv_l = 1.f / l_tot;
-    const long long ob = ((long long)r * a.n_h + head0 + h) * ATT_DC;
+      if (c.last()) {
+        // ---------------------------------------------------------- epilogue of the segment
+        // O is read out before this thread writes the next segment's first P,
+        // which is what PV of that tile (overwriting O) waits for.
+        const SegInfo& S = c.S;
+        float* lred = red + 256;
+        lred[L] = l_run;
+        ok = group_sync(524) && ok;
+        const float l_tot = l_run + lred[L ^ 64];
+        ok = ok && mbar_wait(&pv_done[j & 1], (j >> 1) & 1, abort_flag, 525);
+        tc_fence_after();
+        const float inv_l = 1.f / l_tot;
+        const long long ob = ((long long)S.r * a.n_h + head0 + h) * ATT_DC;
+        const bool direct = S.pslot < 0;
 #pragma unroll 1
-    for (int c = 0; c < 256; c += 16) {
-      float o[16];
-      tmem_ld32<16>(tO + c + lane_off, o);
-      tmem_wait_ld();
-      if (!ok) continue;
-      // TMEM column c of this lane: latent index 256*(c/128) + 128*g + c%128
-      const int d = 256 * (c >> 7) + 128 * g + (c & 127);
-      if (direct) {
-        uint4 v0 = make_uint4(pack_bf16(o[0] * inv_l, o[1] * inv_l), pack_bf16(o[2] * inv_l, o[3] * inv_l),
-                              pack_bf16(o[4] * inv_l, o[5] * inv_l), pack_bf16(o[6] * inv_l, o[7] * inv_l));
-        uint4 v1 = make_uint4(pack_bf16(o[8] * inv_l, o[9] * inv_l), pack_bf16(o[10] * inv_l, o[11] * inv_l),
-                              pack_bf16(o[12] * inv_l, o[13] * inv_l), pack_bf16(o[14] * inv_l, o[15] * inv_l));
-        uint4* dst = reinterpret_cast<uint4*>(a.o_lat + ob + d);
-        dst[0] = v0;
-        dst[1] = v1;
-      } else {
-        float4* dst = reinterpret_cast<float4*>(a.o_part + (long long)split * a.rows * a.n_h * ATT_DC + ob + d);
+        for (int cc = 0; cc < 256; cc += 16) {
+          float o[16];
+          tmem_ld32<16>(tO + cc + lane_off, o);
+          tmem_wait_ld();
+          if (!ok) continue;
+          // TMEM column cc of this lane: latent index 256*(cc/128) + 128*g + cc%128
+          const int d = 256 * (cc >> 7) + 128 * g + (cc & 127);
+          if (direct) {
+            uint4 v0 = make_uint4(pack_bf16(o[0] * inv_l, o[1] * inv_l), pack_bf16(o[2] * inv_l, o[3] * inv_l),
+                                  pack_bf16(o[4] * inv_l, o[5] * inv_l), pack_bf16(o[6] * inv_l, o[7] * inv_l));
+            uint4 v1 = make_uint4(pack_bf16(o[8] * inv_l, o[9] * inv_l), pack_bf16(o[10] * inv_l, o[11] * inv_l),
+                                  pack_bf16(o[12] * inv_l, o[13] * inv_l), pack_bf16(o[14] * inv_l, o[15] * inv_l));
+            uint4* dst = reinterpret_cast<uint4*>(a.o_lat + ob + d);
+            dst[0] = v0;
+            dst[1] = v1;
+          } else {
+            float4* dst =
+                reinterpret_cast<float4*>(a.o_part + ((long long)S.pslot * a.n_h + head0 + h) * ATT_DC + d);
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          dst[e] = make_float4(o[4 * e] * inv_l, o[4 * e + 1] * inv_l, o[4 * e + 2] * inv_l, o[4 * e + 3] * inv_l);
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_float4(o[4 * e] * inv_l, o[4 * e + 1] * inv_l, o[4 * e + 2] * inv_l,
+                                   o[4 * e + 3] * inv_l);
+          }
+        }
+        tc_fence_before();
+        if (ok && g == 0) {
+          const float lse = (m_run + log2f(l_tot)) * 0.69314718055994531f;
+          if (direct) {
+            if (a.lse) a.lse[(long long)S.r * a.n_h + head0 + h] = lse;
+          } else {
+            a.lse_part[(long long)S.pslot * a.n_h + head0 + h] = lse;
+          }
+        }
       }
-    }
-    if (ok && g == 0) {
-      const float lse = (m_run + log2f(l_tot)) * 0.69314718055994531f;
-      const long long li = (long long)r * a.n_h + head0 + h;
-      if (direct) {
-        if (a.lse) a.lse[li] = lse;
-      } else {
-        a.lse_part[(long long)split * a.rows * a.n_h + li] = lse;
-      }
+      c.step(a);
     }
   }
   tc_fence_before();

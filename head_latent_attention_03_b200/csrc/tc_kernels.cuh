@@ -266,29 +266,75 @@ inline int heads_per_cta(const mla_layer_desc* D) { return D->n_h == 16 ? 16 : 3
 // 128-head layers run on CTA pairs (tc_attn2.cuh), one pair per (row, split)
 inline bool use_pair_kernel(const mla_layer_desc* D) { return D->n_h == 128; }
 
+// Host side of the attention work plan (the device side is
+// mla_attn_plan_kernel).  Automatic decode plans deal the tiles of all rows
+// out to one wave of CTAs (or CTA pairs) in equal contiguous ranges; explicit
+// split counts cut every row into that many segments, one per CTA; prefill
+// (and decode with num_splits == 1) runs one CTA per row with no plan at all.
+// The host bounds the segment and slot counts for the grid and the workspace;
+// the plan kernel fills in the actual lists from kv_len.
 struct AttnPlan {
-  int n_splits, span;
+  bool use_plan;  // false: CTA w = row w, nothing to combine
+  int splits;     // explicit segments per row (> 0) or 0 (automatic)
+  int workers;    // CTAs (CTA pairs) the plan is made for = grid size / head groups
+  int max_units, max_slots;
 };
-inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int requested) {
-  AttnPlan p;
-  // work units in flight per wave: one per SM, or one per SM pair
-  const bool pair = use_pair_kernel(D);
-  const int groups = pair ? 1 : D->n_h / heads_per_cta(D);
-  const long long base = (long long)rows * groups;
-  const long long target = pair ? 2LL * (num_sms() / 2) : 2LL * num_sms();
-  int s = requested;
-  if (s <= 0) s = (int)std::max<long long>(1, (target + base - 1) / base);
-  s = std::max(1, std::min(s, (max_len + ATT_TILE - 1) / ATT_TILE));
-  const int per = (max_len + s - 1) / s;
-  p.span = (per + ATT_TILE - 1) / ATT_TILE * ATT_TILE;
-  p.n_splits = (max_len + p.span - 1) / p.span;
+inline int attn_groups(const mla_layer_desc* D) { return use_pair_kernel(D) ? 1 : D->n_h / heads_per_cta(D); }
+// One wave: one CTA per SM, or one CTA pair per two SMs.
+inline int attn_wave_workers(const mla_layer_desc* D) {
+  return std::max(1, use_pair_kernel(D) ? num_sms() / 2 : num_sms() / attn_groups(D));
+}
+inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int requested, int workers = 0) {
+  AttnPlan p{};
+  const int max_tiles = std::max(1, (max_len + ATT_TILE - 1) / ATT_TILE);
+  if (requested == 1) {
+    p.use_plan = false;
+    p.splits = 1;
+    p.workers = rows;
+    return p;
+  }
+  p.use_plan = true;
+  if (requested > 1) {
+    p.splits = std::min(requested, max_tiles);
+    p.max_units = rows * p.splits;
+    p.workers = p.max_units;
+    p.max_slots = p.splits > 1 ? p.max_units : 0;
+    return p;
+  }
+  p.splits = 0;
+  p.workers = workers > 0 ? workers : attn_wave_workers(D);
+  // each range boundary cuts at most one row: segments <= rows + workers - 1,
+  // and the segments of cut rows number at most 2 * (workers - 1)
+  p.max_units = rows + p.workers;
+  p.max_slots = std::min(p.max_units, 2 * p.workers);
   return p;
 }
-inline size_t ws_attn(const mla_layer_desc* D, int rows, int max_len, int n_splits) {
-  if (n_splits <= 1) return 0;
+// Workspace carve of one plan: segment list, row table, CTA table, partials.
+struct AttnWs {
+  int4* units;
+  int4* row_info;
+  int* work;
+  int* n_units;
+  float* o_part;
+  float* lse_part;
+};
+inline bool carve_attn(Carver& c, const mla_layer_desc* D, int rows, const AttnPlan& p, AttnWs* w) {
+  *w = AttnWs{};
+  if (!p.use_plan) return true;
+  w->units = (int4*)c.take((size_t)p.max_units * sizeof(int4));
+  w->row_info = (int4*)c.take((size_t)rows * sizeof(int4));
+  w->work = (int*)c.take((size_t)(p.workers + 1) * sizeof(int));
+  w->n_units = (int*)c.take(16);
+  if (p.max_slots > 0) {
+    w->o_part = (float*)c.take((size_t)p.max_slots * D->n_h * ATT_DC * 4);
+    w->lse_part = (float*)c.take((size_t)p.max_slots * D->n_h * 4);
+  }
+  return c.ok();
+}
+inline size_t ws_attn(const mla_layer_desc* D, int rows, const AttnPlan& p) {
   Carver c{nullptr, 0};
-  c.take((size_t)n_splits * rows * D->n_h * ATT_DC * 4);
-  c.take((size_t)n_splits * rows * D->n_h * 4);
+  AttnWs w;
+  carve_attn(c, D, rows, p, &w);
   return c.used;
 }
 
@@ -301,9 +347,9 @@ static size_t tc_workspace_size(const mla_layer_desc* D, int T, int B, int max_k
   if (T > 0) w = std::max({ws_compress(D, T), ws_absorb(D, T), ws_out(D, T)});
   if (B > 0 && max_kv_len > 0) {
     const int max_len = (max_kv_len + 63) / 64 * 64;
-    const AttnPlan p = plan_attn(D, B, max_len, 0);
-    const int s = std::max(p.n_splits, std::min(16, (max_len + ATT_TILE - 1) / ATT_TILE));
-    w = std::max(w, ws_attn(D, B, max_len, s));
+    // the automatic plan, or any explicit split count up to 16
+    w = std::max(w, ws_attn(D, B, plan_attn(D, B, max_len, 0)));
+    w = std::max(w, ws_attn(D, B, plan_attn(D, B, max_len, 16)));
   }
   return w + 256;
 }
@@ -493,19 +539,21 @@ static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, con
 static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
                                  const mla_paged_cache* cache, const int32_t* kv_len, const int32_t* q_start,
                                  int q_per_seq, int rows, void* ws, size_t ws_bytes, int num_splits, void* o_lat,
-                                 float* lse, cudaStream_t st) {
+                                 float* lse, cudaStream_t st, int workers = 0) {
   if (!aligned16(q_lat) || !aligned16(q_rope) || !aligned16(cache->pool) || !aligned16(o_lat))
     return MLA_ERR_INVALID_ARG;
   const int H = heads_per_cta(D);
   const int max_len = cache->max_blocks * 64;
-  const AttnPlan p = plan_attn(D, rows, max_len, kv_len ? num_splits : 1);
+  const AttnPlan p = plan_attn(D, rows, max_len, kv_len ? num_splits : 1, workers);
   Carver cv = carve(ws, ws_bytes);
-  float* o_part = nullptr;
-  float* lse_part = nullptr;
-  if (p.n_splits > 1) {
-    o_part = (float*)cv.take((size_t)p.n_splits * rows * D->n_h * ATT_DC * 4);
-    lse_part = (float*)cv.take((size_t)p.n_splits * rows * D->n_h * 4);
-    if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  AttnWs aw{};
+  if (p.use_plan && (!ws || !carve_attn(cv, D, rows, p, &aw))) return MLA_ERR_CAPACITY;
+  if (p.use_plan) {
+    MLA_COUNT_LAUNCH();
+    mla_attn_plan_kernel<<<1, 1024, 0, st>>>(kv_len, q_start, q_per_seq, rows, max_len, p.workers, p.splits,
+                                             p.max_units, p.max_slots, aw.units, aw.row_info, aw.work,
+                                             aw.n_units);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }
   const bool pair = use_pair_kernel(D);
   const uint32_t q_box = pair ? 64u : (uint32_t)H;  // query rows per CTA
@@ -518,18 +566,19 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   a.n_h = D->n_h;
   a.rows = rows;
   a.q_per_seq = q_per_seq;
-  a.span = p.span;
-  a.n_splits = p.n_splits;
   a.num_blocks = cache->num_blocks;
   a.max_blocks = cache->max_blocks;
   a.scale_log2 = (float)(D->attn_logit_factor / sqrt((double)(D->d_h + D->d_hr)) * 1.4426950408889634);
   a.table = cache->block_table;
+  a.pool = (const uint8_t*)cache->pool;
   a.kv_len = kv_len;
   a.q_start = q_start;
   a.o_lat = (__nv_bfloat16*)o_lat;
   a.lse = lse;
-  a.o_part = o_part;
-  a.lse_part = lse_part;
+  a.units = aw.units;
+  a.work = aw.work;
+  a.o_part = aw.o_part;
+  a.lse_part = aw.lse_part;
   cudaError_t e;
   if (pair) {
     CUtensorMap m1, m2, m8;
@@ -537,19 +586,19 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
         !map_cache_chunks(&m2, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 2) ||
         !map_cache_chunks(&m8, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 8))
       return MLA_ERR_CUDA;
-    dim3 grid(2 * p.n_splits, 1, rows);
+    dim3 grid(2 * p.workers);
     cudaFuncSetAttribute(mla_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
     MLA_COUNT_LAUNCH();
     mla_attn_pair_kernel<<<grid, PairCfg::THREADS, PairCfg::SMEM, st>>>(mq, mr, m1, m2, m8, a);
     e = cudaGetLastError();
   } else {
-    dim3 grid(p.n_splits, D->n_h / H, rows);
+    dim3 grid(p.workers * attn_groups(D));
     e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
-  if (p.n_splits > 1) {
+  if (p.max_slots > 0) {
     MLA_COUNT_LAUNCH();
-    mla_combine_kernel<<<rows * D->n_h, 128, 0, st>>>(o_part, lse_part, p.n_splits, rows, D->n_h,
+    mla_combine_kernel<<<rows * D->n_h, 128, 0, st>>>(aw.o_part, aw.lse_part, aw.row_info, D->n_h,
                                                       (__nv_bfloat16*)o_lat, lse);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   }

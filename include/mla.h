@@ -129,7 +129,13 @@ mla_status_t mla_absorb_q(const mla_layer_desc* desc, const mla_weights* w,
  *   q_lat [B, n_h, d_c], q_rope [B, n_h, d_hr]
  *   kv_len [B] int32     rows attended by sequence b (including the token just
  *                        appended), 1 <= kv_len[b] <= max_blocks*block_size
- *   num_splits           KV splits per sequence; 0 = chosen from the SM count
+ *   num_splits           how the KV rows are cut into work units:
+ *                        0 = automatic: all sequences' 128-row tiles are
+ *                        spread over about two waves of equal units (a
+ *                        sequence is cut only where it is longer than a
+ *                        unit); S > 0 = every sequence cut into min(S, its
+ *                        tiles) parts.  Cut sequences are merged by a
+ *                        log-sum-exp combine.  1 needs no workspace.
  *   o_lat [B, n_h, d_c]  out: softmax-weighted sum of c^KV (desc dtype)
  *   lse   [B, n_h] float out (may be NULL): natural-log sum of exp(s_j)      */
 mla_status_t mla_decode_attn(const mla_layer_desc* desc, const void* q_lat, const void* q_rope,
@@ -145,11 +151,12 @@ mla_status_t mla_decode_attn(const mla_layer_desc* desc, const void* q_lat, cons
  * plug-in that may not touch the host framework's allocator) and that has no
  * spare buffer to lend as workspace.
  * Same arguments and results as mla_decode_attn, minus the workspace.  The
- * split partials live in a library-owned device array of 32 MiB
- * (every device that loads the library holds it until the process exits);
- * with num_splits == 0 the automatic split count is lowered until the
- * partials fit, an explicit num_splits whose partials need more than 32 MiB
- * (num_splits * B * n_h * 2052 bytes, bf16 layers) returns MLA_ERR_CAPACITY,
+ * work-unit list and split partials live in a library-owned device array of
+ * 32 MiB (every device that loads the library holds it until the process
+ * exits); with num_splits == 0 the automatic plan uses fewer, longer units
+ * until they fit, an explicit num_splits whose unit list and partials need
+ * more than 32 MiB (about num_splits * B * (n_h * 2052 + 16) bytes, bf16
+ * layers) returns MLA_ERR_CAPACITY,
  * as does an fp32 layer whose score scratch (B * n_h * max_blocks *
  * block_size * 4 bytes) exceeds it.  No device memory is allocated or freed.
  * The first call on a device looks up the array's address on that device (a
