@@ -1,35 +1,76 @@
-// tc_gemm.cuh — weight-streaming bf16 GEMM on the 5th-generation tensor cores.
+// tc_gemm.cuh — weight-streaming bf16 GEMM on the 5th-generation tensor cores,
+// with the K-split reduction and the projection's epilogue fused in.
 //
-//   P[ks][z][t][n] = sum_{k in split ks} A_z[n][k] * X_z[t][k]      (fp32)
+//   Y[z][t][n] = epilogue( sum_k A_z[n][k] * X_z[t][k] )
 //
 // A holds weight rows (output features n, on the MMA's M = 128), X holds the
 // token activations (tokens t on the MMA's N).  Putting the weights on M keeps
 // the 128-lane accumulator full at decode batch sizes (T = 32 or 64 tokens),
 // where every projection of the MLA layer is bound by streaming its weights.
-// One CTA computes one 128 x TN tile over one K split:
+//
+// A tile's K range is split over the S CTAs of one thread-block cluster
+// (S <= 8), so that a wave of CTAs covers the GPU even when a projection has
+// few 128-row tiles.  Each CTA accumulates its K slice in TMEM, parks the fp32
+// tile in its own shared memory, and after a cluster barrier CTA s sums rows
+// [128 s / S, 128 (s+1) / S) of all S tiles over distributed shared memory, in
+// rank order (deterministic), and applies the epilogue: bf16 or fp32 store,
+// RoPE of the decoupled key/query features, or the paged-cache scatter of
+// [c^KV | k^R].  No partial sums reach global memory.
+//
+// Warps (192 threads):
 //   warp 0      TMA producer (A and X tiles, 64-wide K chunks, SW128)
 //   warp 1      MMA issuer (one elected thread) and TMEM owner
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator, fp32 stores
+//   warps 2..5  TMEM -> shared memory; all six warps share the reduction
+// Launched with programmatic stream serialisation: the weight tiles of the
+// first pipeline stages are requested before pdl_wait(), i.e. while the
+// previous kernel of the step is still finishing; activations are read and
+// outputs written only after it.
 // A is K-major ([n][k] rows) or, for the per-head absorbed W^UK, MN-major
 // (memory [k][n], n contiguous).  Two weight segments (e.g. W^DKV and W^KR)
 // can share one launch: M tiles below m_tiles0 read map A0, the rest A1.
 #pragma once
 
 #include "common.cuh"
+#include "rope.cuh"
 
 namespace mla {
+
+enum GemmEpiKind : int {
+  EPI_F32 = 0,    // fp32 y[z][t][n]
+  EPI_BF16 = 1,   // bf16 y[z][t][n]
+  EPI_CACHE = 2,  // features [0, d_c): c^KV; [d_c, d_c + d_hr): RoPE_pos(k^R); bf16 into the paged cache
+  EPI_Q = 3,      // features [0, nq): q^C (bf16 [t][nq]); [nq, nq + n_h d_hr): RoPE_pos(q^R) (bf16)
+};
+
+struct GemmEpi {
+  int kind;
+  void* out;                 // EPI_F32 / EPI_BF16
+  long long out_z, out_t;    // element strides of y (feature stride 1)
+  RopeParams rp;             // EPI_CACHE / EPI_Q
+  const int32_t* pos;        // [T]
+  int d_hr;
+  // EPI_CACHE
+  int d_c;
+  const int32_t* seq_idx;    // [T]
+  __nv_bfloat16* pool;
+  int num_blocks, max_blocks, block_size;
+  const int32_t* table;
+  // EPI_Q
+  int nq, n_h;
+  __nv_bfloat16* q_c;
+  __nv_bfloat16* q_rope;
+};
 
 struct GemmArgs {
   int k_chunks;        // K / 64 (whole contraction)
   int k_chunks_split;  // chunks per split
-  int n_tiles;         // token tiles
+  int splits;          // CTAs per cluster (K splits of one tile)
   int m_tiles0;        // M tiles of segment 0
   int n_out0, n_out1;  // rows of segment 0 / segment 1 (n_out1 = 0: one segment)
   int T;               // tokens
   int a_z_rows;        // per-batch row offset into A (K-major: output rows; MN-major: K rows)
   int b_z_cols;        // per-batch column offset into X
-  float* out;          // fp32 partials
-  long long out_split, out_z, out_t;  // element strides (feature stride is 1)
+  GemmEpi e;
 };
 
 constexpr int GEMM_THREADS = 192;
@@ -40,13 +81,68 @@ struct GemmCfg {
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
   static constexpr int B_BYTES = TN * GEMM_BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int NST = (196 * 1024 / STAGE) < 6 ? (196 * 1024 / STAGE) : 6;
+  // up to two CTAs per SM for TN <= 64 (about 110 KB each), one otherwise
+  static constexpr int BUDGET = TN <= 64 ? 104 * 1024 : 200 * 1024;
+  static constexpr int NST = (BUDGET / STAGE) < 8 ? (BUDGET / STAGE) : 8;
+  static constexpr int RED_BYTES = TN * GEMM_BM * 4;     // fp32 tile, [t][row]
   static constexpr int TMEM_COLS = TN <= 32 ? 32 : TN <= 64 ? 64 : TN <= 128 ? 128 : 256;
   static constexpr int SMEM = NST * STAGE + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int CTAS_PER_SM = TN <= 64 ? 2 : 1;
+  static_assert(RED_BYTES <= NST * STAGE, "the reduction tile reuses the pipeline stages");
 };
 
+// Final value of features (n, n+1) of token t in batch z.
+__device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, int n, float2 v) {
+  switch (e.kind) {
+    case EPI_F32:
+      *reinterpret_cast<float2*>(reinterpret_cast<float*>(e.out) + z * e.out_z + t * e.out_t + n) = v;
+      break;
+    case EPI_BF16:
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(e.out) + z * e.out_z + t * e.out_t + n) =
+          __floats2bfloat162_rn(v.x, v.y);
+      break;
+    case EPI_CACHE: {
+      const int row = e.d_c + e.d_hr;
+      const long long p = e.pos[t];
+      if (n >= e.d_c) {
+        float c, s;
+        rope_cos_sin(e.rp, e.d_hr, (n - e.d_c) / 2, p, &c, &s);
+        const float a = v.x, b = v.y;
+        v.x = a * c - b * s;
+        v.y = a * s + b * c;
+      }
+      const int page = (int)(p / e.block_size);
+      const int blk = (page >= 0 && page < e.max_blocks) ? e.table[(long long)e.seq_idx[t] * e.max_blocks + page] : -1;
+      if (blk < 0 || blk >= e.num_blocks) {
+        if (n == 0) record_error(ERR_CAPACITY, 301);
+        break;
+      }
+      __nv_bfloat16* dst = e.pool + ((long long)blk * e.block_size + p % e.block_size) * row + n;
+      *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(v.x, v.y);
+      break;
+    }
+    case EPI_Q: {
+      if (n < e.nq) {
+        *reinterpret_cast<__nv_bfloat162*>(e.q_c + (long long)t * e.nq + n) = __floats2bfloat162_rn(v.x, v.y);
+        break;
+      }
+      const int r = n - e.nq;  // = head * d_hr + 2k
+      float c, s;
+      rope_cos_sin(e.rp, e.d_hr, (r % e.d_hr) / 2, e.pos[t], &c, &s);
+      const float a = v.x, b = v.y;
+      *reinterpret_cast<__nv_bfloat162*>(e.q_rope + (long long)t * e.n_h * e.d_hr + r) =
+          __floats2bfloat162_rn(a * c - b * s, a * s + b * c);
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+// Grid: x = M tile * splits + split (clusters of `splits` along x), y = token
+// tile, z = batch.
 template <int TN, bool A_MN>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
+__global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                      const __grid_constant__ CUtensorMap mB, const GemmArgs g) {
   using C = GemmCfg<TN>;
@@ -59,12 +155,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* done = empty + C::NST;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(smem);  // [TN][128] fp32 after the main loop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x;
-  const int nt = blockIdx.y % g.n_tiles, ks = blockIdx.y / g.n_tiles, z = blockIdx.z;
+  const int S = g.splits;
+  const int mt = blockIdx.x / S, ks = blockIdx.x % S;  // ks = rank in the cluster
+  const int nt = blockIdx.y, z = blockIdx.z;
   const int kc0 = ks * g.k_chunks_split;
-  const int nk = min(g.k_chunks_split, g.k_chunks - kc0);
+  const int nk = max(0, min(g.k_chunks_split, g.k_chunks - kc0));
   const bool seg1 = mt >= g.m_tiles0;
   const CUtensorMap* mA = seg1 ? &mA1 : &mA0;
   const int m_row0 = (seg1 ? mt - g.m_tiles0 : mt) * GEMM_BM;  // first row inside the segment
@@ -83,25 +181,40 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();  // after the TMEM allocation: a dependent CTA on this SM allocates after it
 
+  bool ok = true;
   if (warp == 0) {
     if (elect_one()) {
       tma_prefetch_desc(mA);
       tma_prefetch_desc(&mB);
-      for (int i = 0; i < nk; ++i) {
-        const int s = i % C::NST;
-        if (i >= C::NST && !mbar_wait(&empty[s], ((i / C::NST) - 1) & 1, abort_flag, 201)) break;
-        uint8_t* sa = smem + s * C::STAGE;
-        uint8_t* sb = sa + C::A_BYTES;
-        mbar_expect_tx(&full[s], C::STAGE);
+      auto load_a = [&](int i, uint8_t* sa) {
         const int kx = (kc0 + i) * GEMM_BK;
         if (!A_MN) {
-          tma_load_2d(sa, mA, &full[s], kx, z * g.a_z_rows + m_row0);
+          tma_load_2d(sa, mA, &full[i % C::NST], kx, z * g.a_z_rows + m_row0);
         } else {
-          tma_load_2d(sa, mA, &full[s], m_row0, z * g.a_z_rows + kx);
-          tma_load_2d(sa + 8192, mA, &full[s], m_row0 + 64, z * g.a_z_rows + kx);
+          tma_load_2d(sa, mA, &full[i % C::NST], m_row0, z * g.a_z_rows + kx);
+          tma_load_2d(sa + 8192, mA, &full[i % C::NST], m_row0 + 64, z * g.a_z_rows + kx);
         }
-        tma_load_2d(sb, &mB, &full[s], z * g.b_z_cols + kx, nt * TN);
+      };
+      auto load_b = [&](int i, uint8_t* sb) {
+        tma_load_2d(sb, &mB, &full[i % C::NST], z * g.b_z_cols + (kc0 + i) * GEMM_BK, nt * TN);
+      };
+      // weights of the first stages: they depend on no earlier kernel
+      const int pre = min(nk, C::NST);
+      for (int i = 0; i < pre; ++i) {
+        mbar_expect_tx(&full[i], C::STAGE);
+        load_a(i, smem + i * C::STAGE);
+      }
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) load_b(i, smem + i * C::STAGE + C::A_BYTES);
+      for (int i = pre; i < nk; ++i) {
+        const int s = i % C::NST;
+        if (!mbar_wait(&empty[s], ((i / C::NST) - 1) & 1, abort_flag, 201)) break;
+        uint8_t* sa = smem + s * C::STAGE;
+        mbar_expect_tx(&full[s], C::STAGE);
+        load_a(i, sa);
+        load_b(i, sa + C::A_BYTES);
       }
     }
   } else if (warp == 1) {
@@ -125,125 +238,61 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mma_commit(done);
     }
   } else {
-    // epilogue warps 2..5: warp w reads TMEM lanes 32*(w%4) .. +31
+    // TMEM -> shared memory: warp w reads TMEM lanes 32*(w%4) .. +31 (tile rows)
     const int q = warp & 3;
-    const int row = q * 32 + lane;  // output feature inside the tile
-    const int n_seg = seg1 ? g.n_out1 : g.n_out0;
-    const int n_in_seg = m_row0 + row;
-    const int n_out = (seg1 ? g.n_out0 : 0) + n_in_seg;
-    const bool ok = mbar_wait(done, 0, abort_flag, 203) && nk > 0;
+    const int row = q * 32 + lane;
+    ok = mbar_wait(done, 0, abort_flag, 203);
     tc_fence_after();
-    float* dst = g.out + (long long)ks * g.out_split + (long long)z * g.out_z + n_out;
 #pragma unroll 1
     for (int c0 = 0; c0 < TN; c0 += 16) {
       float v[16];
       tmem_ld32<16>(tmem + ((uint32_t)(q * 32) << 16) + c0, v);
       tmem_wait_ld();
-      if (ok && n_in_seg < n_seg) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = nt * TN + c0 + j;
-          if (t < g.T) dst[(long long)t * g.out_t] = v[j];
-        }
-      }
+      for (int j = 0; j < 16; ++j) red[(c0 + j) * GEMM_BM + row] = nk > 0 ? v[j] : 0.f;
     }
   }
+  __syncwarp();
+  tc_fence_before();
+  // every CTA of the cluster has its partial tile in shared memory
+  if (S > 1)
+    cluster_sync_all();
+  else
+    __syncthreads();
+  ok = __syncthreads_and(ok ? 1 : 0) != 0;
+  pdl_wait();  // outputs may be read by the previous kernel until it has finished
+
+  // this CTA's rows of the tile, summed over the cluster in rank order
+  const int r0 = ((ks * GEMM_BM) / S) & ~1, r1 = ks == S - 1 ? GEMM_BM : (((ks + 1) * GEMM_BM) / S) & ~1;
+  const int n_pairs = (r1 - r0) / 2;
+  const int n_seg = seg1 ? g.n_out1 : g.n_out0;
+  const uint32_t red_addr = smem_u32(red);
+  if (ok) {
+    for (int e = threadIdx.x; e < n_pairs * TN; e += GEMM_THREADS) {
+      const int t_loc = e / n_pairs, rr = r0 + 2 * (e % n_pairs);
+      const int t = nt * TN + t_loc;
+      const int n_in_seg = m_row0 + rr;
+      if (t >= g.T || n_in_seg >= n_seg) continue;
+      const uint32_t off = (uint32_t)(t_loc * GEMM_BM + rr) * 4u;
+      float2 v;
+      if (S == 1) {
+        v = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(red) + off);
+      } else {
+        v = make_float2(0.f, 0.f);
+        for (int sr = 0; sr < S; ++sr) {
+          const float2 p = ld_cluster_f2(mapa_shared(red_addr + off, (uint32_t)sr));
+          v.x += p.x;
+          v.y += p.y;
+        }
+      }
+      gemm_epilogue(g.e, z, t, (seg1 ? g.n_out0 : 0) + n_in_seg, v);
+    }
+  }
+  // keep this CTA's tile alive until every CTA of the cluster has read it
+  if (S > 1) cluster_sync_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
-}
-
-// ---------------------------------------------------------------------------
-// finishing kernels: sum the K splits (fixed order, deterministic) and apply
-// the step's epilogue.  Each thread owns one adjacent pair of features so that
-// a RoPE pair (2k, 2k+1) stays in one thread.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float2 sum_splits(const float* p, int splits, long long split_stride) {
-  float2 a = *reinterpret_cast<const float2*>(p);
-  for (int s = 1; s < splits; ++s) {
-    const float2 b = *reinterpret_cast<const float2*>(p + s * split_stride);
-    a.x += b.x;
-    a.y += b.y;
-  }
-  return a;
-}
-
-// compress_append: [c^KV | RoPE_pos(k^R)] -> bf16 cache slot of (seq_idx[t], pos[t]).
-__global__ void finish_compress_kernel(const float* __restrict__ part, int splits, long long split_stride, int T,
-                                       int d_c, int d_hr, RopeParams rp, const int32_t* __restrict__ seq_idx,
-                                       const int32_t* __restrict__ pos, __nv_bfloat16* __restrict__ pool,
-                                       int num_blocks, const int32_t* __restrict__ table, int max_blocks,
-                                       int block_size) {
-  const int row = d_c + d_hr;
-  const int pairs = row / 2;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)T * pairs) return;
-  const int t = (int)(idx / pairs), e = 2 * (int)(idx % pairs);
-  float2 v = sum_splits(part + (long long)t * row + e, splits, split_stride);
-  const long long p = pos[t];
-  if (e >= d_c) {
-    float c, s;
-    rope_cos_sin(rp, d_hr, (e - d_c) / 2, p, &c, &s);
-    const float a = v.x, b = v.y;
-    v.x = a * c - b * s;
-    v.y = a * s + b * c;
-  }
-  const int page = (int)(p / block_size);
-  const int blk = (page >= 0 && page < max_blocks) ? table[(long long)seq_idx[t] * max_blocks + page] : -1;
-  if (blk < 0 || blk >= num_blocks) {
-    if (e == 0) record_error(ERR_CAPACITY, 301);
-    return;
-  }
-  __nv_bfloat16* dst = pool + ((long long)blk * block_size + p % block_size) * row + e;
-  *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(v.x, v.y);
-}
-
-// plain conversion: y[z][t][n] (bf16) = sum of splits, n < n_out.
-__global__ void finish_bf16_kernel(const float* __restrict__ part, int splits, long long split_stride, int Z, int T,
-                                   int n_out, long long in_z, long long in_t, __nv_bfloat16* __restrict__ y,
-                                   long long y_z, long long y_t) {
-  const int pairs = n_out / 2;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)Z * T * pairs) return;
-  const int e = 2 * (int)(idx % pairs);
-  const long long zt = idx / pairs;
-  const int t = (int)(zt % T), z = (int)(zt / T);
-  const float2 v = sum_splits(part + z * in_z + t * in_t + e, splits, split_stride);
-  *reinterpret_cast<__nv_bfloat162*>(y + z * y_z + t * y_t + e) = __floats2bfloat162_rn(v.x, v.y);
-}
-
-// absorb_q second projection: features [0, nq) are q^C (bf16 copy), features
-// [nq, nq + n_h*d_hr) are q^R of head (n-nq)/d_hr, rotated at pos[t].
-__global__ void finish_q_kernel(const float* __restrict__ part, int splits, long long split_stride, int T, int nq,
-                                int n_h, int d_hr, RopeParams rp, const int32_t* __restrict__ pos,
-                                __nv_bfloat16* __restrict__ q_c, __nv_bfloat16* __restrict__ q_rope) {
-  const int n_all = nq + n_h * d_hr;
-  const int pairs = n_all / 2;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)T * pairs) return;
-  const int t = (int)(idx / pairs), e = 2 * (int)(idx % pairs);
-  float2 v = sum_splits(part + (long long)t * n_all + e, splits, split_stride);
-  if (e < nq) {
-    *reinterpret_cast<__nv_bfloat162*>(q_c + (long long)t * nq + e) = __floats2bfloat162_rn(v.x, v.y);
-    return;
-  }
-  const int r = e - nq;  // = head * d_hr + 2k
-  float c, s;
-  rope_cos_sin(rp, d_hr, (r % d_hr) / 2, pos[t], &c, &s);
-  const float a = v.x, b = v.y;
-  *reinterpret_cast<__nv_bfloat162*>(q_rope + (long long)t * n_h * d_hr + r) =
-      __floats2bfloat162_rn(a * c - b * s, a * s + b * c);
-}
-
-// fp32 output: u[t][n] = sum of splits.
-__global__ void finish_f32_kernel(const float* __restrict__ part, int splits, long long split_stride, int T,
-                                  int n_out, float* __restrict__ u) {
-  const int pairs = n_out / 2;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)T * pairs) return;
-  const int t = (int)(idx / pairs), e = 2 * (int)(idx % pairs);
-  const float2 v = sum_splits(part + (long long)t * n_out + e, splits, split_stride);
-  *reinterpret_cast<float2*>(u + (long long)t * n_out + e) = v;
 }
 
 }  // namespace mla

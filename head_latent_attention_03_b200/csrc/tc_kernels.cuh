@@ -10,6 +10,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <utility>
 
 #include "../../include/mla.h"
 #include "common.cuh"
@@ -112,21 +113,53 @@ struct Carver {
 // ---------------------------------------------------------------------------
 // GEMM planning and launch
 // ---------------------------------------------------------------------------
+// Launch with programmatic stream serialisation (the kernel calls pdl_wait()
+// before it touches anything an earlier kernel writes) and, for cluster > 1,
+// a thread-block cluster of that many CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  int n = 0;
+  at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    at[n].id = cudaLaunchAttributeClusterDimension;
+    at[n].val.clusterDim.x = (unsigned)cluster;
+    at[n].val.clusterDim.y = 1;
+    at[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = at;
+  cfg.numAttrs = n;
+  MLA_COUNT_LAUNCH();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 struct GemmPlan {
   int tn, n_tiles, splits, kcs;
 };
 
 inline int pick_tn(int T) { return T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256; }
+inline int gemm_ctas_per_sm(int tn) { return tn <= 64 ? GemmCfg<64>::CTAS_PER_SM : 1; }
 
+// K splits per tile (= cluster size, at most 8) so that the launch fills one
+// wave of the GPU's CTA slots.
 inline GemmPlan plan_gemm(int m_tiles, int Z, int T, int K) {
   GemmPlan p;
   p.tn = pick_tn(T);
   p.n_tiles = (T + p.tn - 1) / p.tn;
   const int kc = K / GEMM_BK;
   const long long tiles = (long long)m_tiles * p.n_tiles * Z;
-  const int want = (int)std::max<long long>(1, (2LL * num_sms() + tiles - 1) / tiles);
-  const int cap_traffic = std::max(1, K / (8 * std::max(T, 1)));  // fp32 partials <= 1/4 of weight bytes
-  int s = std::min({want, cap_traffic, std::max(1, kc / 2)});
+  const long long slots = (long long)num_sms() * gemm_ctas_per_sm(p.tn);
+  int s = (int)std::max<long long>(1, std::min<long long>(8, slots / std::max<long long>(tiles, 1)));
+  s = std::max(1, std::min(s, kc / 2));
   p.kcs = (kc + s - 1) / s;
   p.splits = (kc + p.kcs - 1) / p.kcs;
   return p;
@@ -138,9 +171,7 @@ inline cudaError_t launch_gemm_t(const CUtensorMap& A0, const CUtensorMap& A1, c
   auto kfn = gemm_bf16_kernel<TN, A_MN>;
   constexpr int smem = GemmCfg<TN>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  MLA_COUNT_LAUNCH();
-  kfn<<<grid, GEMM_THREADS, smem, st>>>(A0, A1, B, g);
-  return cudaGetLastError();
+  return launch_pdl(kfn, grid, dim3(GEMM_THREADS), smem, st, g.splits, A0, A1, B, g);
 }
 
 template <bool A_MN>
@@ -154,7 +185,7 @@ inline cudaError_t launch_gemm_tn(int tn, const CUtensorMap& A0, const CUtensorM
   }
 }
 
-// One projection: out[ks][z][t][n] over two weight segments (rows0 of A0,
+// One projection: Y = epilogue(A X) over two weight segments (rows0 of A0,
 // rows1 of A1), K contraction, Z batches.
 struct GemmCall {
   const void* a0;
@@ -169,8 +200,7 @@ struct GemmCall {
   int K, T, Z, a_z_rows, b_z_cols;
 };
 
-inline mla_status_t run_gemm(const GemmCall& c, float* out, long long out_z, long long out_t, long long out_split,
-                             const GemmPlan& p, cudaStream_t st) {
+inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan& p, cudaStream_t st) {
   CUtensorMap A0, A1, B;
   bool ok;
   if (!c.a_mn) {
@@ -187,22 +217,19 @@ inline mla_status_t run_gemm(const GemmCall& c, float* out, long long out_z, lon
   GemmArgs g;
   g.k_chunks = c.K / GEMM_BK;
   g.k_chunks_split = p.kcs;
-  g.n_tiles = p.n_tiles;
+  g.splits = p.splits;
   g.m_tiles0 = (c.rows0 + GEMM_BM - 1) / GEMM_BM;
   g.n_out0 = c.rows0;
   g.n_out1 = c.a1 ? c.rows1 : 0;
   g.T = c.T;
   g.a_z_rows = c.a_z_rows;
   g.b_z_cols = c.b_z_cols;
-  g.out = out;
-  g.out_split = out_split;
-  g.out_z = out_z;
-  g.out_t = out_t;
+  g.e = e;
   const int m_tiles = g.m_tiles0 + (c.a1 ? (c.rows1 + GEMM_BM - 1) / GEMM_BM : 0);
-  dim3 grid(m_tiles, p.n_tiles * p.splits, c.Z);
-  const cudaError_t e = c.a_mn ? launch_gemm_tn<true>(p.tn, A0, A1, B, g, grid, st)
-                               : launch_gemm_tn<false>(p.tn, A0, A1, B, g, grid, st);
-  return e == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  dim3 grid(m_tiles * p.splits, p.n_tiles, c.Z);
+  const cudaError_t err = c.a_mn ? launch_gemm_tn<true>(p.tn, A0, A1, B, g, grid, st)
+                                 : launch_gemm_tn<false>(p.tn, A0, A1, B, g, grid, st);
+  return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 inline unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
@@ -234,31 +261,18 @@ inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
   return plan_gemm((D->d + 127) / 128, 1, T, D->n_h * D->d_h);
 }
 
-inline size_t ws_compress(const mla_layer_desc* D, int T) {
-  Carver c{nullptr, 0};
-  c.take((size_t)plan_compress(D, T).splits * T * (D->d_c + D->d_hr) * 4);
-  return c.used;
-}
+// Workspace of the projections: only the bf16 intermediates between two
+// GEMMs (K splits are reduced inside each GEMM's cluster).
+inline size_t ws_compress(const mla_layer_desc*, int) { return 0; }
 inline size_t ws_absorb(const mla_layer_desc* D, int T) {
   Carver c{nullptr, 0};
-  const int nq = D->n_h * D->d_h;
-  if (D->d_cq) {
-    c.take((size_t)T * D->d_cq * 2);
-  }
-  c.take((size_t)T * nq * 2);
-  size_t part = 0;
-  if (D->d_cq) part = std::max(part, (size_t)plan_q1(D, T).splits * T * D->d_cq * 4);
-  part = std::max(part, (size_t)plan_q2(D, T).splits * T * (nq + D->n_h * D->d_hr) * 4);
-  part = std::max(part, (size_t)plan_q3(D, T).splits * D->n_h * T * D->d_c * 4);
-  c.take(part);
+  if (D->d_cq) c.take((size_t)T * D->d_cq * 2);
+  c.take((size_t)T * D->n_h * D->d_h * 2);
   return c.used;
 }
 inline size_t ws_out(const mla_layer_desc* D, int T) {
   Carver c{nullptr, 0};
   c.take((size_t)T * D->n_h * D->d_h * 2);
-  size_t part = std::max((size_t)plan_o1(D, T).splits * D->n_h * T * D->d_h * 4,
-                         (size_t)plan_o2(D, T).splits * T * D->d * 4);
-  c.take(part);
   return c.used;
 }
 
@@ -363,14 +377,11 @@ static Carver carve(void* ws, size_t ws_bytes) {
 
 static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weights* w, const void* h,
                                        const int32_t* seq_idx, const int32_t* pos, int T, mla_paged_cache* cache,
-                                       void* ws, size_t ws_bytes, cudaStream_t st) {
+                                       void*, size_t, cudaStream_t st) {
   if (!aligned16(h) || !aligned16(w->w_dkv) || !aligned16(w->w_kr) || !aligned16(cache->pool))
     return MLA_ERR_INVALID_ARG;
-  Carver cv = carve(ws, ws_bytes);
-  const int row = D->d_c + D->d_hr;
-  const GemmPlan p = plan_compress(D, T);
-  float* part = (float*)cv.take((size_t)p.splits * T * row * 4);
-  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  // [c^KV ; k^R] = [W^DKV ; W^KR] h  (eq 9 + decoupled key), RoPE on k^R,
+  // bf16 rows scattered into the paged cache
   GemmCall c{};
   c.a0 = w->w_dkv;
   c.rows0 = D->d_c;
@@ -383,14 +394,19 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   c.K = D->d;
   c.T = T;
   c.Z = 1;
-  mla_status_t s = run_gemm(c, part, 0, row, (long long)T * row, p, st);
-  if (s != MLA_OK) return s;
-  const long long n = (long long)T * row / 2;
-  MLA_COUNT_LAUNCH();
-  finish_compress_kernel<<<blocks_for(n, 256), 256, 0, st>>>(
-      part, p.splits, (long long)T * row, T, D->d_c, D->d_hr, rope_of(D), seq_idx, pos,
-      (__nv_bfloat16*)cache->pool, cache->num_blocks, cache->block_table, cache->max_blocks, D->block_size);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  GemmEpi e{};
+  e.kind = EPI_CACHE;
+  e.rp = rope_of(D);
+  e.pos = pos;
+  e.d_hr = D->d_hr;
+  e.d_c = D->d_c;
+  e.seq_idx = seq_idx;
+  e.pool = (__nv_bfloat16*)cache->pool;
+  e.num_blocks = cache->num_blocks;
+  e.max_blocks = cache->max_blocks;
+  e.block_size = D->block_size;
+  e.table = cache->block_table;
+  return run_gemm(c, e, plan_compress(D, T), st);
 }
 
 static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos,
@@ -403,12 +419,6 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
   const int q_in = D->d_cq ? D->d_cq : D->d;
   __nv_bfloat16* cq = D->d_cq ? (__nv_bfloat16*)cv.take((size_t)T * D->d_cq * 2) : nullptr;
   __nv_bfloat16* qc = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
-  const GemmPlan p1 = D->d_cq ? plan_q1(D, T) : GemmPlan{};
-  const GemmPlan p2 = plan_q2(D, T), p3 = plan_q3(D, T);
-  size_t part_bytes = (size_t)p2.splits * T * (nq + nr) * 4;
-  part_bytes = std::max(part_bytes, (size_t)p3.splits * D->n_h * T * D->d_c * 4);
-  if (D->d_cq) part_bytes = std::max(part_bytes, (size_t)p1.splits * T * D->d_cq * 4);
-  float* part = (float*)cv.take(part_bytes);
   if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   mla_status_t s;
   const void* qsrc = h;
@@ -423,11 +433,11 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.K = D->d;
     c.T = T;
     c.Z = 1;
-    if ((s = run_gemm(c, part, 0, D->d_cq, (long long)T * D->d_cq, p1, st)) != MLA_OK) return s;
-    const long long n = (long long)T * D->d_cq / 2;
-    MLA_COUNT_LAUNCH();
-    finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p1.splits, (long long)T * D->d_cq, 1, T, D->d_cq, 0,
-                                                            D->d_cq, cq, 0, D->d_cq);
+    GemmEpi e{};
+    e.kind = EPI_BF16;
+    e.out = cq;
+    e.out_t = D->d_cq;
+    if ((s = run_gemm(c, e, plan_q1(D, T), st)) != MLA_OK) return s;
     qsrc = cq;
   }
   {  // [q^C ; q^R] = [W^UQ ; W^QR] c^Q   (eq 13 + decoupled query), RoPE on q^R
@@ -443,11 +453,16 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.K = q_in;
     c.T = T;
     c.Z = 1;
-    if ((s = run_gemm(c, part, 0, nq + nr, (long long)T * (nq + nr), p2, st)) != MLA_OK) return s;
-    const long long n = (long long)T * (nq + nr) / 2;
-    MLA_COUNT_LAUNCH();
-    finish_q_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p2.splits, (long long)T * (nq + nr), T, nq, D->n_h,
-                                                         D->d_hr, rope_of(D), pos, qc, (__nv_bfloat16*)q_rope);
+    GemmEpi e{};
+    e.kind = EPI_Q;
+    e.rp = rope_of(D);
+    e.pos = pos;
+    e.d_hr = D->d_hr;
+    e.nq = nq;
+    e.n_h = D->n_h;
+    e.q_c = qc;
+    e.q_rope = (__nv_bfloat16*)q_rope;
+    if ((s = run_gemm(c, e, plan_q2(D, T), st)) != MLA_OK) return s;
   }
   {  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major
     GemmCall c{};
@@ -464,16 +479,14 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.Z = D->n_h;
     c.a_z_rows = D->d_h;
     c.b_z_cols = D->d_h;
-    // part[ks][head][t][c] ; q_lat[t][head][c]
-    if ((s = run_gemm(c, part, (long long)T * D->d_c, D->d_c, (long long)D->n_h * T * D->d_c, p3, st)) != MLA_OK)
-      return s;
-    const long long n = (long long)D->n_h * T * D->d_c / 2;
-    MLA_COUNT_LAUNCH();
-    finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p3.splits, (long long)D->n_h * T * D->d_c, D->n_h,
-                                                            T, D->d_c, (long long)T * D->d_c, D->d_c,
-                                                            (__nv_bfloat16*)q_lat, D->d_c, (long long)D->n_h * D->d_c);
+    GemmEpi e{};  // q_lat[t][head][c]
+    e.kind = EPI_BF16;
+    e.out = q_lat;
+    e.out_z = D->d_c;
+    e.out_t = (long long)D->n_h * D->d_c;
+    if ((s = run_gemm(c, e, plan_q3(D, T), st)) != MLA_OK) return s;
   }
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return MLA_OK;
 }
 
 static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, const void* o_lat, int T, float* u,
@@ -482,8 +495,6 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
   Carver cv = carve(ws, ws_bytes);
   const int nq = D->n_h * D->d_h;
   __nv_bfloat16* o = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
-  const GemmPlan p1 = plan_o1(D, T), p2 = plan_o2(D, T);
-  float* part = (float*)cv.take(std::max((size_t)p1.splits * D->n_h * T * D->d_h * 4, (size_t)p2.splits * T * D->d * 4));
   if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   mla_status_t s;
   {  // o_i = W^UV_i o_lat_i  (eq 11 absorbed): per head, A = W^UV_i [d_h, d_c]
@@ -499,12 +510,12 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
     c.Z = D->n_h;
     c.a_z_rows = D->d_h;
     c.b_z_cols = D->d_c;
-    if ((s = run_gemm(c, part, (long long)T * D->d_h, D->d_h, (long long)D->n_h * T * D->d_h, p1, st)) != MLA_OK)
-      return s;
-    const long long n = (long long)D->n_h * T * D->d_h / 2;
-    MLA_COUNT_LAUNCH();
-    finish_bf16_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p1.splits, (long long)D->n_h * T * D->d_h, D->n_h,
-                                                            T, D->d_h, (long long)T * D->d_h, D->d_h, o, D->d_h, nq);
+    GemmEpi e{};  // o[t][head][d_h]
+    e.kind = EPI_BF16;
+    e.out = o;
+    e.out_z = D->d_h;
+    e.out_t = nq;
+    if ((s = run_gemm(c, e, plan_o1(D, T), st)) != MLA_OK) return s;
   }
   {  // u = W^O o   (eq 8)
     GemmCall c{};
@@ -517,12 +528,13 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
     c.K = nq;
     c.T = T;
     c.Z = 1;
-    if ((s = run_gemm(c, part, 0, D->d, (long long)T * D->d, p2, st)) != MLA_OK) return s;
-    const long long n = (long long)T * D->d / 2;
-    MLA_COUNT_LAUNCH();
-    finish_f32_kernel<<<blocks_for(n, 256), 256, 0, st>>>(part, p2.splits, (long long)T * D->d, T, D->d, u);
+    GemmEpi e{};
+    e.kind = EPI_F32;
+    e.out = u;
+    e.out_t = D->d;
+    if ((s = run_gemm(c, e, plan_o2(D, T), st)) != MLA_OK) return s;
   }
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return MLA_OK;
 }
 
 template <int H>
