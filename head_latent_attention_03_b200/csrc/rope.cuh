@@ -40,4 +40,31 @@ __device__ inline void rope_cos_sin(const RopeParams& rp, int d_hr, int k, long 
   rope_cos_sin_theta(rope_theta(rp, d_hr, k), pos, c, s);
 }
 
+// Frequencies theta_k of one layer, computed once on the host (fp64).
+constexpr int ROPE_MAX_PAIRS = 64;
+struct RopeTable {
+  double theta[ROPE_MAX_PAIRS];
+};
+inline RopeTable rope_table(const RopeParams& rp, int d_hr) {
+  RopeTable t{};
+  for (int k = 0; k < d_hr / 2 && k < ROPE_MAX_PAIRS; ++k) t.theta[k] = rope_theta(rp, d_hr, k);
+  return t;
+}
+
+// cos/sin of pos * theta for the bf16 path: the angle is formed in fp64 and
+// reduced modulo 2 pi with Cody and Waite's two-constant scheme (2 pi split
+// into a double head and the double nearest to the remainder), then the
+// reduced angle in [-pi, pi] is evaluated in fp32.  Absolute error about
+// 3e-7, far below bf16 resolution, at a fraction of an fp64 sincos.
+__device__ inline void rope_cos_sin_reduced(double theta, long long pos, float* c, float* s) {
+  constexpr double kTwoPiHead = 6.283185307179586;        // 2 pi rounded to double
+  constexpr double kTwoPiTail = 2.4492935982947064e-16;   // 2 pi - kTwoPiHead
+  constexpr double kInvTwoPi = 0.15915494309189535;       // 1 / (2 pi)
+  const double a = (double)pos * theta;
+  const double n = rint(a * kInvTwoPi);
+  double r = fma(-n, kTwoPiHead, a);
+  r = fma(-n, kTwoPiTail, r);
+  sincosf((float)r, s, c);
+}
+
 }  // namespace mla

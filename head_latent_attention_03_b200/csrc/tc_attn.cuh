@@ -176,6 +176,8 @@ __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const i
   __shared__ int s_lastw[1024];
   __shared__ int s_per;
   const int tid = threadIdx.x, nt = blockDim.x;
+  pdl_trigger();
+  pdl_wait();  // kv_len may come from the previous kernel; the workspace may still be in its use
   auto kv_of = [&](int b) -> int {
     const int kv = kv_len ? kv_len[b] : q_start[b / q_per_seq] + b % q_per_seq + 1;
     return min(max(kv, 0), max_len);
@@ -312,7 +314,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // worker run side by side and share its cache tiles in L2
   const int n_grp = a.n_h / H;
   const int worker = blockIdx.x / n_grp, grp = blockIdx.x % n_grp;
-  const int2 range = att_work(a, worker);
   const int head0 = grp * H;
 
   if (threadIdx.x == 0) {
@@ -340,6 +341,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();  // after the TMEM allocation
+  pdl_wait();     // the plan, the queries and the cache come from earlier kernels
+  // nothing written by an earlier kernel is read above this line
+  const int2 range = att_work(a, worker);
   const uint32_t tS = tmem;            // S^T buffers at columns [0, 2H)
   const uint32_t tO = tmem + 2 * H;    // O^T M-block m at columns 2H + m*H
 
@@ -716,6 +721,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 __global__ void mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                                    const int4* __restrict__ row_info, int n_h, __nv_bfloat16* __restrict__ o_lat,
                                    float* __restrict__ lse) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x / n_h, h = blockIdx.x % n_h;
   const int4 info = row_info[r];
   const int n_parts = info.y, slot0 = info.z;

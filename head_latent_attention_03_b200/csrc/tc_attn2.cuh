@@ -103,7 +103,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   // both CTAs of the pair walk the same segment list
   const int worker = blockIdx.x >> 1;
-  const int2 range = att_work(a, worker);
   const int head0 = (int)rank * 64;
   const int tunit = rank == 0 ? worker : -1;  // trace slot (leader only)
   (void)tunit;
@@ -134,6 +133,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   cluster_sync_all();  // peer barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_trigger();  // after the TMEM allocation
+  pdl_wait();     // the plan, the queries and the cache come from earlier kernels
+  // nothing written by an earlier kernel is read above this line
+  const int2 range = att_work(a, worker);
   if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 0, 0);
   const uint32_t tS = tmem;         // S buffers: columns [0,64) and [64,128)
   const uint32_t tO = tmem + 128;   // O: columns [128,256) (d_c 0..255) and [256,384) (256..511)

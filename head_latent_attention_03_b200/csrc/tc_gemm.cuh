@@ -21,10 +21,9 @@
 //   warp 0      TMA producer (A and X tiles, 64-wide K chunks, SW128)
 //   warp 1      MMA issuer (one elected thread) and TMEM owner
 //   warps 2..5  TMEM -> shared memory; all six warps share the reduction
-// Launched with programmatic stream serialisation: the weight tiles of the
-// first pipeline stages are requested before pdl_wait(), i.e. while the
-// previous kernel of the step is still finishing; activations are read and
-// outputs written only after it.
+// Launched with programmatic stream serialisation: set-up and an L2 prefetch
+// of the first weight tiles overlap the previous kernel of the step; every
+// load into shared memory and every output store waits for it.
 // A is K-major ([n][k] rows) or, for the per-head absorbed W^UK, MN-major
 // (memory [k][n], n contiguous).  Two weight segments (e.g. W^DKV and W^KR)
 // can share one launch: M tiles below m_tiles0 read map A0, the rest A1.
@@ -46,7 +45,7 @@ struct GemmEpi {
   int kind;
   void* out;                 // EPI_F32 / EPI_BF16
   long long out_z, out_t;    // element strides of y (feature stride 1)
-  RopeParams rp;             // EPI_CACHE / EPI_Q
+  RopeTable rope;            // EPI_CACHE / EPI_Q: theta_k of the layer
   const int32_t* pos;        // [T]
   int d_hr;
   // EPI_CACHE
@@ -106,7 +105,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
       const long long p = e.pos[t];
       if (n >= e.d_c) {
         float c, s;
-        rope_cos_sin(e.rp, e.d_hr, (n - e.d_c) / 2, p, &c, &s);
+        rope_cos_sin_reduced(e.rope.theta[(n - e.d_c) / 2], p, &c, &s);
         const float a = v.x, b = v.y;
         v.x = a * c - b * s;
         v.y = a * s + b * c;
@@ -128,7 +127,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
       }
       const int r = n - e.nq;  // = head * d_hr + 2k
       float c, s;
-      rope_cos_sin(e.rp, e.d_hr, (r % e.d_hr) / 2, e.pos[t], &c, &s);
+      rope_cos_sin_reduced(e.rope.theta[(r % e.d_hr) / 2], e.pos[t], &c, &s);
       const float a = v.x, b = v.y;
       *reinterpret_cast<__nv_bfloat162*>(e.q_rope + (long long)t * e.n_h * e.d_hr + r) =
           __floats2bfloat162_rn(a * c - b * s, a * s + b * c);
@@ -200,14 +199,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
       auto load_b = [&](int i, uint8_t* sb) {
         tma_load_2d(sb, &mB, &full[i % C::NST], z * g.b_z_cols + (kc0 + i) * GEMM_BK, nt * TN);
       };
-      // weights of the first stages: they depend on no earlier kernel
+      // While the previous kernel finishes, pull this CTA's first weight
+      // tiles into L2; every load into shared memory waits for it.
       const int pre = min(nk, C::NST);
+      for (int i = 0; i < pre; ++i) {
+        const int kx = (kc0 + i) * GEMM_BK;
+        if (!A_MN) {
+          tma_prefetch_l2_2d(mA, kx, z * g.a_z_rows + m_row0);
+        } else {
+          tma_prefetch_l2_2d(mA, m_row0, z * g.a_z_rows + kx);
+          tma_prefetch_l2_2d(mA, m_row0 + 64, z * g.a_z_rows + kx);
+        }
+      }
+      pdl_wait();
       for (int i = 0; i < pre; ++i) {
         mbar_expect_tx(&full[i], C::STAGE);
         load_a(i, smem + i * C::STAGE);
+        load_b(i, smem + i * C::STAGE + C::A_BYTES);
       }
-      pdl_wait();
-      for (int i = 0; i < pre; ++i) load_b(i, smem + i * C::STAGE + C::A_BYTES);
       for (int i = pre; i < nk; ++i) {
         const int s = i % C::NST;
         if (!mbar_wait(&empty[s], ((i / C::NST) - 1) & 1, abort_flag, 201)) break;

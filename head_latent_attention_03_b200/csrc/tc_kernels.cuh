@@ -396,7 +396,7 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   c.Z = 1;
   GemmEpi e{};
   e.kind = EPI_CACHE;
-  e.rp = rope_of(D);
+  e.rope = rope_table(rope_of(D), D->d_hr);
   e.pos = pos;
   e.d_hr = D->d_hr;
   e.d_c = D->d_c;
@@ -455,7 +455,7 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.Z = 1;
     GemmEpi e{};
     e.kind = EPI_Q;
-    e.rp = rope_of(D);
+    e.rope = rope_table(rope_of(D), D->d_hr);
     e.pos = pos;
     e.d_hr = D->d_hr;
     e.nq = nq;
@@ -543,9 +543,7 @@ static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, con
   auto kfn = mla_attn_kernel<H>;
   constexpr int smem = AttnCfg<H>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  MLA_COUNT_LAUNCH();
-  kfn<<<grid, ATT_THREADS, smem, st>>>(mq, mr, mc, a);
-  return cudaGetLastError();
+  return launch_pdl(kfn, grid, dim3(ATT_THREADS), smem, st, 1, mq, mr, mc, a);
 }
 
 static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
@@ -561,11 +559,11 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   AttnWs aw{};
   if (p.use_plan && (!ws || !carve_attn(cv, D, rows, p, &aw))) return MLA_ERR_CAPACITY;
   if (p.use_plan) {
-    MLA_COUNT_LAUNCH();
-    mla_attn_plan_kernel<<<1, 1024, 0, st>>>(kv_len, q_start, q_per_seq, rows, max_len, p.workers, p.splits,
-                                             p.max_units, p.max_slots, aw.units, aw.row_info, aw.work,
-                                             aw.n_units);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    const int threads = std::min(1024, std::max(32, (rows + 31) / 32 * 32));
+    if (launch_pdl(mla_attn_plan_kernel, dim3(1), dim3(threads), 0, st, 1, kv_len, q_start, q_per_seq, rows,
+                   max_len, p.workers, p.splits, p.max_units, p.max_slots, aw.units, aw.row_info, aw.work,
+                   aw.n_units) != cudaSuccess)
+      return MLA_ERR_CUDA;
   }
   const bool pair = use_pair_kernel(D);
   const uint32_t q_box = pair ? 64u : (uint32_t)H;  // query rows per CTA
@@ -600,19 +598,18 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
       return MLA_ERR_CUDA;
     dim3 grid(2 * p.workers);
     cudaFuncSetAttribute(mla_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
-    MLA_COUNT_LAUNCH();
-    mla_attn_pair_kernel<<<grid, PairCfg::THREADS, PairCfg::SMEM, st>>>(mq, mr, m1, m2, m8, a);
-    e = cudaGetLastError();
+    // cluster dimensions are compiled in (__cluster_dims__)
+    e = launch_pdl(mla_attn_pair_kernel, grid, dim3(PairCfg::THREADS), PairCfg::SMEM, st, 1, mq, mr, m1, m2, m8, a);
   } else {
     dim3 grid(p.workers * attn_groups(D));
     e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (p.max_slots > 0) {
-    MLA_COUNT_LAUNCH();
-    mla_combine_kernel<<<rows * D->n_h, 128, 0, st>>>(aw.o_part, aw.lse_part, aw.row_info, D->n_h,
-                                                      (__nv_bfloat16*)o_lat, lse);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if (launch_pdl(mla_combine_kernel, dim3(rows * D->n_h), dim3(128), 0, st, 1, (const float*)aw.o_part,
+                   (const float*)aw.lse_part, (const int4*)aw.row_info, D->n_h, (__nv_bfloat16*)o_lat, lse) !=
+        cudaSuccess)
+      return MLA_ERR_CUDA;
   }
   return MLA_OK;
 }
