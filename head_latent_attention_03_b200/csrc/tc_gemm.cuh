@@ -75,18 +75,30 @@ struct GemmArgs {
 constexpr int GEMM_THREADS = 192;
 constexpr int GEMM_BM = 128, GEMM_BK = 64;
 
-template <int TN>
+#ifndef MLA_GEMM_KC
+#define MLA_GEMM_KC 1  // 64-column K chunks per weight TMA box (K-major weights)
+#endif
+
+// A stage holds KC consecutive 64-wide K chunks of the weight tile and of the
+// activations, each fetched by one TMA box (rows x KC chunks).  DEEP: one CTA
+// per SM with up to 8 stages in flight (projections whose tiles fit one wave
+// of SMs); otherwise two CTAs per SM with about 100 KB each (projections with
+// more tiles than SMs).
+template <int TN, int KC, bool DEEP>
 struct GemmCfg {
-  static constexpr int A_BYTES = GEMM_BM * GEMM_BK * 2;  // 16 KB
-  static constexpr int B_BYTES = TN * GEMM_BK * 2;
+  static constexpr int A_CHUNK = GEMM_BM * GEMM_BK * 2;  // 16 KB
+  static constexpr int B_CHUNK = TN * GEMM_BK * 2;
+  static constexpr int A_BYTES = KC * A_CHUNK;
+  static constexpr int B_BYTES = KC * B_CHUNK;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  // up to two CTAs per SM for TN <= 64 (about 110 KB each), one otherwise
-  static constexpr int BUDGET = TN <= 64 ? 104 * 1024 : 200 * 1024;
+  static constexpr bool TWO = !DEEP && TN <= 64 && 2 * STAGE <= 104 * 1024;
+  static constexpr int BUDGET = TWO ? 104 * 1024 : 200 * 1024;
   static constexpr int NST = (BUDGET / STAGE) < 8 ? (BUDGET / STAGE) : 8;
   static constexpr int RED_BYTES = TN * GEMM_BM * 4;     // fp32 tile, [t][row]
   static constexpr int TMEM_COLS = TN <= 32 ? 32 : TN <= 64 ? 64 : TN <= 128 ? 128 : 256;
   static constexpr int SMEM = NST * STAGE + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int CTAS_PER_SM = TN <= 64 ? 2 : 1;
+  static constexpr int CTAS_PER_SM = TWO ? 2 : 1;
+  static_assert(NST >= 2, "pipeline depth");
   static_assert(RED_BYTES <= NST * STAGE, "the reduction tile reuses the pipeline stages");
 };
 
@@ -140,12 +152,13 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
 
 // Grid: x = M tile * splits + split (clusters of `splits` along x), y = token
 // tile, z = batch.
-template <int TN, bool A_MN>
-__global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
+template <int TN, bool A_MN, int KC, bool DEEP>
+__global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_SM)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
                      const __grid_constant__ CUtensorMap mB, const GemmArgs g) {
-  using C = GemmCfg<TN>;
+  using C = GemmCfg<TN, KC, DEEP>;
   static_assert(TN % 16 == 0 && TN >= 16 && TN <= 256, "token tile");
+  static_assert(!A_MN || KC == 1, "MN-major weights load one chunk per stage");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -187,28 +200,31 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
     if (elect_one()) {
       tma_prefetch_desc(mA);
       tma_prefetch_desc(&mB);
+      // stage i covers chunks [kc0 + KC i, kc0 + KC (i+1)); chunks past this
+      // split's range are fetched (or zero-filled past K) but not multiplied
+      const int ns = (nk + KC - 1) / KC;
       auto load_a = [&](int i, uint8_t* sa) {
-        const int kx = (kc0 + i) * GEMM_BK;
+        const int kc = kc0 + i * KC;
         if (!A_MN) {
-          tma_load_2d(sa, mA, &full[i % C::NST], kx, z * g.a_z_rows + m_row0);
+          tma_load_3d(sa, mA, &full[i % C::NST], 0, z * g.a_z_rows + m_row0, kc);
         } else {
-          tma_load_2d(sa, mA, &full[i % C::NST], m_row0, z * g.a_z_rows + kx);
-          tma_load_2d(sa + 8192, mA, &full[i % C::NST], m_row0 + 64, z * g.a_z_rows + kx);
+          tma_load_2d(sa, mA, &full[i % C::NST], m_row0, z * g.a_z_rows + kc * GEMM_BK);
+          tma_load_2d(sa + 8192, mA, &full[i % C::NST], m_row0 + 64, z * g.a_z_rows + kc * GEMM_BK);
         }
       };
       auto load_b = [&](int i, uint8_t* sb) {
-        tma_load_2d(sb, &mB, &full[i % C::NST], z * g.b_z_cols + (kc0 + i) * GEMM_BK, nt * TN);
+        tma_load_3d(sb, &mB, &full[i % C::NST], 0, nt * TN, z * g.b_z_cols / GEMM_BK + kc0 + i * KC);
       };
       // While the previous kernel finishes, pull this CTA's first weight
       // tiles into L2; every load into shared memory waits for it.
-      const int pre = min(nk, C::NST);
+      const int pre = min(ns, C::NST);
       for (int i = 0; i < pre; ++i) {
-        const int kx = (kc0 + i) * GEMM_BK;
+        const int kc = kc0 + i * KC;
         if (!A_MN) {
-          tma_prefetch_l2_2d(mA, kx, z * g.a_z_rows + m_row0);
+          tma_prefetch_l2_3d(mA, 0, z * g.a_z_rows + m_row0, kc);
         } else {
-          tma_prefetch_l2_2d(mA, m_row0, z * g.a_z_rows + kx);
-          tma_prefetch_l2_2d(mA, m_row0 + 64, z * g.a_z_rows + kx);
+          tma_prefetch_l2_2d(mA, m_row0, z * g.a_z_rows + kc * GEMM_BK);
+          tma_prefetch_l2_2d(mA, m_row0 + 64, z * g.a_z_rows + kc * GEMM_BK);
         }
       }
       pdl_wait();
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
         load_a(i, smem + i * C::STAGE);
         load_b(i, smem + i * C::STAGE + C::A_BYTES);
       }
-      for (int i = pre; i < nk; ++i) {
+      for (int i = pre; i < ns; ++i) {
         const int s = i % C::NST;
         if (!mbar_wait(&empty[s], ((i / C::NST) - 1) & 1, abort_flag, 201)) break;
         uint8_t* sa = smem + s * C::STAGE;
@@ -229,18 +245,22 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
   } else if (warp == 1) {
     if (elect_one()) {
       const uint32_t idesc = idesc_bf16_f32(GEMM_BM, TN, A_MN, false);
-      for (int i = 0; i < nk; ++i) {
+      const int ns = (nk + KC - 1) / KC;
+      for (int i = 0; i < ns; ++i) {
         const int s = i % C::NST;
         if (!mbar_wait(&full[s], (i / C::NST) & 1, abort_flag, 202)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + s * C::STAGE);
         const uint32_t sb = sa + C::A_BYTES;
+        const int nc = min(KC, nk - i * KC);
+        for (int c = 0; c < nc; ++c) {
 #pragma unroll
-        for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-          const uint64_t ad = A_MN ? smem_desc(sa + kk * 2048, 8192, 1024, SW128)
-                                   : smem_desc(sa + kk * 32, 16, 1024, SW128);
-          const uint64_t bd = smem_desc(sb + kk * 32, 16, 1024, SW128);
-          mma_bf16_ss(tmem, ad, bd, idesc, (i | kk) != 0);
+          for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc(sa + kk * 2048, 8192, 1024, SW128)
+                                     : smem_desc(sa + c * C::A_CHUNK + kk * 32, 16, 1024, SW128);
+            const uint64_t bd = smem_desc(sb + c * C::B_CHUNK + kk * 32, 16, 1024, SW128);
+            mma_bf16_ss(tmem, ad, bd, idesc, (i | c | kk) != 0);
+          }
         }
         mma_commit(&empty[s]);
       }
@@ -277,24 +297,44 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN>::CTAS_PER_SM)
   const int n_seg = seg1 ? g.n_out1 : g.n_out0;
   const uint32_t red_addr = smem_u32(red);
   if (ok) {
-    for (int e = threadIdx.x; e < n_pairs * TN; e += GEMM_THREADS) {
-      const int t_loc = e / n_pairs, rr = r0 + 2 * (e % n_pairs);
-      const int t = nt * TN + t_loc;
-      const int n_in_seg = m_row0 + rr;
-      if (t >= g.T || n_in_seg >= n_seg) continue;
-      const uint32_t off = (uint32_t)(t_loc * GEMM_BM + rr) * 4u;
-      float2 v;
-      if (S == 1) {
-        v = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(red) + off);
-      } else {
-        v = make_float2(0.f, 0.f);
-        for (int sr = 0; sr < S; ++sr) {
-          const float2 p = ld_cluster_f2(mapa_shared(red_addr + off, (uint32_t)sr));
-          v.x += p.x;
-          v.y += p.y;
+    // E elements per thread and round: all their S remote loads are issued
+    // before any is summed, so the DSMEM latency is paid once per round
+    constexpr int E = 4, SMAX = 8;
+    const int n_el = n_pairs * TN;
+    for (int e0 = threadIdx.x; e0 < n_el; e0 += E * GEMM_THREADS) {
+      float2 part[E][SMAX];
+      uint32_t off[E];
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const int e = e0 + q * GEMM_THREADS;
+        const int t_loc = e / n_pairs, rr = r0 + 2 * (e % n_pairs);
+        off[q] = (uint32_t)(t_loc * GEMM_BM + rr) * 4u;
+        if (e >= n_el) continue;
+        if (S == 1) {
+          part[q][0] = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(red) + off[q]);
+        } else {
+#pragma unroll
+          for (int sr = 0; sr < SMAX; ++sr)
+            if (sr < S) part[q][sr] = ld_cluster_f2(mapa_shared(red_addr + off[q], (uint32_t)sr));
         }
       }
-      gemm_epilogue(g.e, z, t, (seg1 ? g.n_out0 : 0) + n_in_seg, v);
+#pragma unroll
+      for (int q = 0; q < E; ++q) {
+        const int e = e0 + q * GEMM_THREADS;
+        if (e >= n_el) continue;
+        const int t_loc = e / n_pairs, rr = r0 + 2 * (e % n_pairs);
+        const int t = nt * TN + t_loc;
+        const int n_in_seg = m_row0 + rr;
+        if (t >= g.T || n_in_seg >= n_seg) continue;
+        float2 v = part[q][0];
+#pragma unroll
+        for (int sr = 1; sr < SMAX; ++sr)
+          if (sr < S) {
+            v.x += part[q][sr].x;
+            v.y += part[q][sr].y;
+          }
+        gemm_epilogue(g.e, z, t, (seg1 ? g.n_out0 : 0) + n_in_seg, v);
+      }
     }
   }
   // keep this CTA's tile alive until every CTA of the cluster has read it

@@ -93,6 +93,23 @@ inline bool map_cache_chunks(CUtensorMap* m, const void* pool, int num_blocks, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A row-major bf16 matrix (`rows` rows of `inner` elements, rows `row_bytes`
+// apart) as a 3D map {column in chunk, row, 64-column chunk}: a box of
+// box_rows rows x kc chunks lands chunk-major (each chunk box_rows x 128 B,
+// 128-byte swizzle), i.e. exactly kc consecutive 2D boxes of 64 columns.
+inline bool map_rows_chunks(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                            uint32_t box_rows, uint32_t kc) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {64, rows, inner / 64};
+  cuuint64_t strides[2] = {row_bytes, 128};
+  cuuint32_t box[3] = {64, box_rows, kc};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---------------------------------------------------------------------------
@@ -144,44 +161,50 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 
 struct GemmPlan {
   int tn, n_tiles, splits, kcs;
+  bool deep;  // one deep-pipelined CTA per SM (else two per SM)
 };
 
 inline int pick_tn(int T) { return T <= 32 ? 32 : T <= 64 ? 64 : T <= 128 ? 128 : 256; }
-inline int gemm_ctas_per_sm(int tn) { return tn <= 64 ? GemmCfg<64>::CTAS_PER_SM : 1; }
+inline int gemm_kc(bool a_mn) { return a_mn ? 1 : MLA_GEMM_KC; }
 
-// K splits per tile (= cluster size, at most 8) so that the launch fills one
-// wave of the GPU's CTA slots.
-inline GemmPlan plan_gemm(int m_tiles, int Z, int T, int K) {
+// Tiles that fit one wave of SMs run one deep-pipelined CTA per SM, their K
+// split over a cluster of up to 8 CTAs to fill the wave; more tiles than SMs
+// run two CTAs per SM (token tiles of at most 64) with no split.
+inline GemmPlan plan_gemm(int m_tiles, int Z, int T, int K, bool a_mn = false) {
   GemmPlan p;
   p.tn = pick_tn(T);
   p.n_tiles = (T + p.tn - 1) / p.tn;
   const int kc = K / GEMM_BK;
+  const int kcb = gemm_kc(a_mn);  // chunks per stage: splits cover whole stages
   const long long tiles = (long long)m_tiles * p.n_tiles * Z;
-  const long long slots = (long long)num_sms() * gemm_ctas_per_sm(p.tn);
+  const int sms = num_sms();
+  p.deep = tiles <= sms || p.tn > 64;
+  const long long slots = (long long)sms * (p.deep ? 1 : 2);
   int s = (int)std::max<long long>(1, std::min<long long>(8, slots / std::max<long long>(tiles, 1)));
-  s = std::max(1, std::min(s, kc / 2));
-  p.kcs = (kc + s - 1) / s;
+  s = std::max(1, std::min(s, kc / (2 * kcb)));
+  p.kcs = ((kc + s - 1) / s + kcb - 1) / kcb * kcb;
   p.splits = (kc + p.kcs - 1) / p.kcs;
   return p;
 }
 
-template <int TN, bool A_MN>
+template <int TN, bool A_MN, bool DEEP>
 inline cudaError_t launch_gemm_t(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B, const GemmArgs& g,
                                  dim3 grid, cudaStream_t st) {
-  auto kfn = gemm_bf16_kernel<TN, A_MN>;
-  constexpr int smem = GemmCfg<TN>::SMEM;
+  constexpr int KC = A_MN ? 1 : MLA_GEMM_KC;
+  auto kfn = gemm_bf16_kernel<TN, A_MN, KC, DEEP>;
+  constexpr int smem = GemmCfg<TN, KC, DEEP>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   return launch_pdl(kfn, grid, dim3(GEMM_THREADS), smem, st, g.splits, A0, A1, B, g);
 }
 
-template <bool A_MN>
+template <bool A_MN, bool DEEP>
 inline cudaError_t launch_gemm_tn(int tn, const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B,
                                   const GemmArgs& g, dim3 grid, cudaStream_t st) {
   switch (tn) {
-    case 32: return launch_gemm_t<32, A_MN>(A0, A1, B, g, grid, st);
-    case 64: return launch_gemm_t<64, A_MN>(A0, A1, B, g, grid, st);
-    case 128: return launch_gemm_t<128, A_MN>(A0, A1, B, g, grid, st);
-    default: return launch_gemm_t<256, A_MN>(A0, A1, B, g, grid, st);
+    case 32: return launch_gemm_t<32, A_MN, DEEP>(A0, A1, B, g, grid, st);
+    case 64: return launch_gemm_t<64, A_MN, DEEP>(A0, A1, B, g, grid, st);
+    case 128: return launch_gemm_t<128, A_MN, true>(A0, A1, B, g, grid, st);
+    default: return launch_gemm_t<256, A_MN, true>(A0, A1, B, g, grid, st);
   }
 }
 
@@ -203,16 +226,17 @@ struct GemmCall {
 inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan& p, cudaStream_t st) {
   CUtensorMap A0, A1, B;
   bool ok;
+  const uint32_t kc = (uint32_t)gemm_kc(c.a_mn);
   if (!c.a_mn) {
-    ok = map_2d(&A0, c.a0, (uint64_t)c.K, (uint64_t)c.rows0 * c.Z, (uint64_t)c.a_row_elems * 2, 64, 128);
-    ok = ok && map_2d(&A1, c.a1 ? c.a1 : c.a0, (uint64_t)c.K, (uint64_t)(c.a1 ? c.rows1 : c.rows0) * c.Z,
-                      (uint64_t)c.a_row_elems * 2, 64, 128);
+    ok = map_rows_chunks(&A0, c.a0, (uint64_t)c.K, (uint64_t)c.rows0 * c.Z, (uint64_t)c.a_row_elems * 2, 128, kc);
+    ok = ok && map_rows_chunks(&A1, c.a1 ? c.a1 : c.a0, (uint64_t)c.K, (uint64_t)(c.a1 ? c.rows1 : c.rows0) * c.Z,
+                               (uint64_t)c.a_row_elems * 2, 128, kc);
   } else {
     ok = map_2d(&A0, c.a0, (uint64_t)c.rows0, (uint64_t)c.a_mn_rows, (uint64_t)c.a_row_elems * 2, 64, 64);
     A1 = A0;
   }
-  ok = ok && map_2d(&B, c.x, (uint64_t)c.x_row_elems, (uint64_t)c.x_rows, (uint64_t)c.x_row_elems * 2, 64,
-                    (uint32_t)p.tn);
+  ok = ok && map_rows_chunks(&B, c.x, (uint64_t)c.x_row_elems, (uint64_t)c.x_rows, (uint64_t)c.x_row_elems * 2,
+                             (uint32_t)p.tn, kc);
   if (!ok) return MLA_ERR_CUDA;
   GemmArgs g;
   g.k_chunks = c.K / GEMM_BK;
@@ -227,8 +251,13 @@ inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan
   g.e = e;
   const int m_tiles = g.m_tiles0 + (c.a1 ? (c.rows1 + GEMM_BM - 1) / GEMM_BM : 0);
   dim3 grid(m_tiles * p.splits, p.n_tiles, c.Z);
-  const cudaError_t err = c.a_mn ? launch_gemm_tn<true>(p.tn, A0, A1, B, g, grid, st)
-                                 : launch_gemm_tn<false>(p.tn, A0, A1, B, g, grid, st);
+  cudaError_t err;
+  if (c.a_mn)
+    err = p.deep ? launch_gemm_tn<true, true>(p.tn, A0, A1, B, g, grid, st)
+                 : launch_gemm_tn<true, false>(p.tn, A0, A1, B, g, grid, st);
+  else
+    err = p.deep ? launch_gemm_tn<false, true>(p.tn, A0, A1, B, g, grid, st)
+                 : launch_gemm_tn<false, false>(p.tn, A0, A1, B, g, grid, st);
   return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -255,7 +284,9 @@ inline GemmPlan plan_q2(const mla_layer_desc* D, int T) {
   const int q_in = D->d_cq ? D->d_cq : D->d;
   return plan_gemm((D->n_h * D->d_h + 127) / 128 + (D->n_h * D->d_hr + 127) / 128, 1, T, q_in);
 }
-inline GemmPlan plan_q3(const mla_layer_desc* D, int T) { return plan_gemm(D->d_c / 128, D->n_h, T, D->d_h); }
+inline GemmPlan plan_q3(const mla_layer_desc* D, int T) {
+  return plan_gemm(D->d_c / 128, D->n_h, T, D->d_h, /*a_mn=*/true);
+}
 inline GemmPlan plan_o1(const mla_layer_desc* D, int T) { return plan_gemm((D->d_h + 127) / 128, D->n_h, T, D->d_c); }
 inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
   return plan_gemm((D->d + 127) / 128, 1, T, D->n_h * D->d_h);
