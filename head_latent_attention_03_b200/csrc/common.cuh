@@ -336,6 +336,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
+// Arrive on another CTA's barrier with CTA-scope release: enough when the
+// data it announces lives in the arriving CTA's own shared memory or TMEM and
+// is consumed there (the other CTA only issues the 2-SM instruction that
+// reads it), and much cheaper than a cluster-scope release.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx_cluster(uint32_t cl_addr, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cl_addr),
                "r"(bytes)

@@ -21,13 +21,16 @@
 // overwrites its own (already multiplied) pair with the columns it needs from
 // the other page.  So every cached byte crosses into shared memory once per
 // CTA that needs it (104 KB per CTA per tile), and the eight 16 KB pair slots
-// keep two tiles in flight.  The cache is read through a 4D view
-// {column, slot, chunk, block} so that one TMA instruction fetches several
-// 64-column chunks of a page at once: per tile and CTA, one RoPE box, one
-// 8-chunk own-page box and two 2-chunk refill boxes.
+// keep two tiles in flight.  Slots recycle one at a time: the own-page pair
+// for slot s of tile j+2 is loaded as soon as PV(j) has read slot s (a commit
+// per slot), and QK(j+2) starts on the first pair to land, so the chain
+// load -> QK -> refill -> PV overlaps across the four pairs of a tile
+// instead of running tile by tile.  The cache is read through a 4D view
+// {column, slot, chunk, block}: per tile and CTA, one RoPE box and four
+// 2-chunk own-page boxes, plus two 2-chunk refill boxes.
 //
 // Warps (224 threads per CTA):
-//   0    own-page producer (RoPE chunk + the 8 latent chunks per tile)
+//   0    own-page producer (RoPE chunk + four latent pairs per tile)
 //   1    MMA issuer (leader CTA only, one thread) and TMEM owner (both CTAs)
 //   2-5  softmax: thread = (head, page half of the tile)
 //   6    other-page producer: refills the pair slots PV needs once QK is done
@@ -43,12 +46,31 @@
 
 namespace mla {
 
+// Signals from the non-leader CTA to the leader's barriers (S consumed, P
+// written, last tile zeroed) announce data in the signalling CTA's own shared
+// memory / TMEM, consumed by its own tensor core: CTA-scope release and
+// acquire suffice (PAIR_CLUSTER_SCOPE = 1 selects cluster scope).
+#ifndef PAIR_CLUSTER_SCOPE
+#define PAIR_CLUSTER_SCOPE 0
+#endif
+#if PAIR_CLUSTER_SCOPE
+#define PAIR_ARRIVE(a) mbar_arrive_cluster(a)
+#define PAIR_TEST(a, p) mbar_test_cluster(a, p)
+#else
+#define PAIR_ARRIVE(a) mbar_arrive_remote(a)
+#define PAIR_TEST(a, p) mbar_test(a, p)
+#endif
+
 #ifndef PAIR_PREFETCH
 #define PAIR_PREFETCH 1  // tiles of own pages prefetched into L2 ahead of their load
 #endif
 
 struct PairCfg {
+#ifdef MLA_TRACE
+  static constexpr int THREADS = 256;  // + a barrier-observer warp
+#else
   static constexpr int THREADS = 224;
+#endif
   static constexpr int Q_CHUNK = 64 * 128;        // 64 heads x 64 columns
   static constexpr int Q_BYTES = 9 * Q_CHUNK;     // 72 KB
   static constexpr int P_BYTES = 2 * 64 * 128;    // 64 heads x 128 tokens (two SW128 K atoms)
@@ -60,7 +82,7 @@ struct PairCfg {
   static constexpr int OFF_ROPE = OFF_P + P_BYTES;
   static constexpr int OFF_PAIR = OFF_ROPE + ROPE;
   static constexpr int OFF_BAR = OFF_PAIR + NP * PAIR;
-  static constexpr int N_BAR = 2 + 2 * NP + 1 + 1 + 2 + 2 + 1 + 2 + 1 + 1 + 2;
+  static constexpr int N_BAR = 4 * NP + 1 + 1 + 2 + 2 + 1 + 2 + 1 + 1 + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int OFF_RED = OFF_MISC + 16;
   static constexpr int SMEM = OFF_RED + 3 * 128 * 4 + 1024;
@@ -72,19 +94,20 @@ struct PairCfg {
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     mla_attn_pair_kernel(const __grid_constant__ CUtensorMap m_qlat, const __grid_constant__ CUtensorMap m_qrope,
                          const __grid_constant__ CUtensorMap m_page1, const __grid_constant__ CUtensorMap m_page2,
-                         const __grid_constant__ CUtensorMap m_page8, const AttnArgs a) {
+                         const AttnArgs a) {
   using C = PairCfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   // Pair commits per tile: one qk_done per pair slot (QK has read it: the
-  // other CTA may refill it), s_full (S ready; the RoPE slot is free) and
-  // pv_done (the tile's pair slots are free, O is stable).  s_full and
+  // other CTA may refill it), one pv_slot per pair slot (PV has read it: the
+  // next own-page load may overwrite it), s_full (S ready; the RoPE slot is
+  // free) and pv_done (O is stable, the P buffer is free).  s_full and
   // pv_done have one instance per tile parity so that a waiter is never two
   // phases behind.
-  uint64_t* own_full = bar;                   // leader [2]: a tile's own latent chunks landed
-  uint64_t* oth_full = own_full + 2;          // leader [NP]: other-page refill landed
+  uint64_t* own_full = bar;                   // leader [NP]: own-page pair landed in the slot
+  uint64_t* oth_full = own_full + C::NP;      // leader [NP]: other-page refill landed
   uint64_t* qk_done = oth_full + C::NP;       // both [NP]: pair commit once QK has read the slot
   uint64_t* rope_full = qk_done + C::NP;      // leader
   uint64_t* q_full = rope_full + 1;           // leader
@@ -95,6 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   uint64_t* last_ready = pv_done + 2;         // leader: both CTAs zeroed the last tile
   uint64_t* grp_bar = last_ready + 1;         // local: 128 softmax threads
   uint64_t* z_land = grp_bar + 1;             // local [2]: last tile's other-page refills
+  uint64_t* pv_slot = z_land + 2;             // both [NP]: pair commit once PV has read the slot
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [3][128]: tile max x2, final sums
@@ -109,13 +133,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NP; ++i) {
+      mbar_init(&own_full[i], 1);
       mbar_init(&oth_full[i], 1);
       mbar_init(&qk_done[i], 1);
+      mbar_init(&pv_slot[i], 1);
     }
     mbar_init(rope_full, 1);
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&own_full[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 2);
       mbar_init(&pv_done[i], 1);
@@ -161,13 +186,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   // The CTA whose own page is k & 1 keeps its own columns there; the other CTA
   // refills the slot with columns 2*(2*(k>>1) + rank) .. +1 of page k & 1.
 
+#ifdef MLA_TRACE
+  if (warp == 7) {
+    if (lane != 0 || rank != 0) {
+    } else {
+    // trace-only observer: completion times of each tile's first own pair,
+    // first refill and P (leader barriers), polled without blocking anyone
+    TileCursor c;
+    c.init(a, range);
+    while (!c.done() && !*abort_flag) {
+      const int g = c.g, s0 = slot_of(g, 0), u0 = use_of(g, 0);
+      const uint64_t t_start = globaltimer_ns();
+      bool seen_own = false, seen_oth = c.zero(), seen_p = false;
+      while (!(seen_own && seen_oth && seen_p) && globaltimer_ns() - t_start < 2000000ull && !*abort_flag) {
+        if (!seen_own && mbar_test(smem_u32(&own_full[s0]), u0 & 1)) { seen_own = true; MLA_TRACE_EVENT(tunit, 3, g); }
+        if (!seen_oth && mbar_test(smem_u32(&oth_full[s0]), u0 & 1)) { seen_oth = true; MLA_TRACE_EVENT(tunit, 4, g); }
+        if (!seen_p && mbar_test_cluster(smem_u32(p_full), g & 1)) { seen_p = true; MLA_TRACE_EVENT(tunit, 15, g); }
+      }
+      c.step(a);
+    }
+    }
+  } else
+#endif
   if (warp == 0) {
     // ------------------------------------------------------------ own-page producer
     // Per tile two TMA instructions: the RoPE chunk (8 KB) and all eight
     // latent chunks of the own page (64 KB, landing in the tile's four
     // consecutive pair slots); per segment the queries of its row.
     if (elect_one()) {
-      tma_prefetch_desc(&m_page8);
+      tma_prefetch_desc(&m_page2);
       const uint32_t lq = mapa_shared(smem_u32(q_full), 0);
       const uint32_t l_rope = mapa_shared(smem_u32(rope_full), 0);
       // Own pages are prefetched into L2 PAIR_PREFETCH tiles ahead: the TMA
@@ -204,12 +251,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         if (rank == 0) mbar_expect_tx(rope_full, 2 * C::ROPE);
         tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, 8, blk);
         MLA_TRACE_EVENT(tunit, 1, g);
-        // the tile's four pair slots were last used by PV(g-2)
-        if (g >= 2 && !mbar_wait(&pv_done[g & 1], ((g - 2) >> 1) & 1, abort_flag, 504)) break;
-        uint64_t* of = &own_full[g & 1];
-        if (rank == 0) mbar_expect_tx(of, 2 * 4 * C::PAIR);
-        tma_load_4d_pair(smem + C::OFF_PAIR + slot_of(g, 0) * C::PAIR, &m_page8, mapa_shared(smem_u32(of), 0), 0, 0,
-                         0, blk);
+        // the own page pair by pair, each into its slot as soon as PV(g-2)
+        // has read that slot: QK(g) starts on the first pair to land
+        bool ok = true;
+        for (int k = 0; k < 4 && ok; ++k) {
+          const int s = slot_of(g, k), u = use_of(g, k);
+          if (u >= 1 && !mbar_wait(&pv_slot[s], (u - 1) & 1, abort_flag, 504)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(&own_full[s], 2 * C::PAIR);
+          tma_load_4d_pair(smem + C::OFF_PAIR + s * C::PAIR, &m_page2, mapa_shared(smem_u32(&own_full[s]), 0), 0, 0,
+                           2 * k, blk);
+        }
+        if (!ok) break;
         MLA_TRACE_EVENT(tunit, 2, g);
         c.step(a);
       }
@@ -219,6 +274,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     TileCursor c;
     c.init(a, range);
     int nz = 0;  // zero tiles so far (phase of z_land)
+    const int tunit6 = rank == 0 ? worker : 256 + worker;  // trace slot of this CTA's refills
+    (void)tunit6;
     bool ok = true;
     while (ok && !c.done()) {
       const int g = c.g;
@@ -230,6 +287,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           if ((k & 1) == (int)rank) continue;  // kept by this CTA
           ok = mbar_wait(&qk_done[s], u & 1, abort_flag, 505);  // QK(g) has read this pair
           if (!ok) break;
+          MLA_TRACE_EVENT(tunit6, zk == 0 && k < 2 ? 12 : 13, g);
           const int b = page_block(c, c.tok() / 64 + (k & 1));
           const int c0 = 2 * (2 * (k >> 1) + (int)rank);  // columns this CTA multiplies in instruction k >> 1
           uint8_t* dst = smem + C::OFF_PAIR + s * C::PAIR;
@@ -269,7 +327,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive_cluster(mapa_shared(smem_u32(last_ready), 0));
+        if (lane == 0 && ok) PAIR_ARRIVE(mapa_shared(smem_u32(last_ready), 0));
         ++nz;
       }
       c.step(a);
@@ -301,6 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       // Work is issued in batches (a tile's 32 latent QK MMAs at once, PV pair
       // by pair): every barrier probe between MMAs costs issue slots.
       int pv_k = 0;  // next pair of PV(cp)
+      int qk_k = 0;  // next pair of QK(cq)
       int q_seen = -1;  // segment whose queries have landed
       int nz = 0;       // zero tiles passed by PV (phase of last_ready)
       bool sbuf_ok = false, rope_pending = false, p_ok = false, ok = true;
@@ -311,12 +370,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         // PV first: it frees the slots that later tiles' loads wait for
         if (cp.g < cq.g) {
           const int jp = cp.g;
-          if (!p_ok) p_ok = mbar_test_cluster(smem_u32(p_full), jp & 1);
+          if (!p_ok) p_ok = PAIR_TEST(smem_u32(p_full), jp & 1);
           if (p_ok) {
             const bool zero = cp.zero();
             while (pv_k < 4) {
               const int s = slot_of(jp, pv_k), u = use_of(jp, pv_k);
-              const bool ready = zero ? mbar_test_cluster(smem_u32(last_ready), nz & 1)
+              const bool ready = zero ? PAIR_TEST(smem_u32(last_ready), nz & 1)
                                       : mbar_test(smem_u32(&oth_full[s]), u & 1);
               if (!ready) break;
               if (pv_k == 0) MLA_TRACE_EVENT(tunit, 14, jp);
@@ -329,6 +388,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
                 const uint64_t bd = smem_desc(pb + kk * 2048, 8192, 1024, SW128);
                 mma_bf16_pair(tO + 128 * i, ad, bd, id_pv, (cp.j > 0 || p > 0 || kk > 0) ? 1u : 0u);
               }
+              mma_commit_pair(&pv_slot[s]);
               // a zero tile's slots had no refill on oth_full: close that phase
               if (zero) mbar_arrive(&oth_full[s]);
               if ((pv_k & 1) == 0) post_peer_refill(pv_k);
@@ -349,25 +409,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         if (!cq.done()) {
           const int jq = cq.g;
           if (!rope_pending) {
-            if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_test_cluster(smem_u32(&s_free[jq & 1]), ((jq >> 1) - 1) & 1);
+            if (!sbuf_ok) sbuf_ok = jq < 2 || PAIR_TEST(smem_u32(&s_free[jq & 1]), ((jq >> 1) - 1) & 1);
             if (q_seen != cq.n && mbar_test(smem_u32(q_full), cq.n & 1)) q_seen = cq.n;
-            if (sbuf_ok && q_seen == cq.n && mbar_test(smem_u32(&own_full[jq & 1]), (jq >> 1) & 1)) {
-              MLA_TRACE_EVENT(tunit, 6, jq);
+            // the latent chunks pair by pair as their slots land; each pair's
+            // commit lets the other CTA refill that slot
+            while (sbuf_ok && q_seen == cq.n && qk_k < 4) {
+              const int s = slot_of(jq, qk_k);
+              if (!mbar_test(smem_u32(&own_full[s]), use_of(jq, qk_k) & 1)) break;
+              if (qk_k == 0) MLA_TRACE_EVENT(tunit, 6, jq);
               tc_fence_after();
-              // the 8 latent chunks, pair by pair; each pair's commit lets the
-              // other CTA refill that slot
-              for (int k = 0; k < 8; ++k) {
-                const uint32_t kb = pair0 + slot_of(jq, k >> 1) * C::PAIR + (k & 1) * 8192;
+              const uint32_t kb = pair0 + s * C::PAIR;
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int k = 2 * qk_k + h2;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                   const uint64_t ad = smem_desc(q_base + k * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
-                  const uint64_t bd = smem_desc(kb + kk * 32, 16, 1024, SW128);
+                  const uint64_t bd = smem_desc(kb + h2 * 8192 + kk * 32, 16, 1024, SW128);
                   mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qk, (k | kk) != 0 ? 1u : 0u);
                 }
-                if (k & 1) mma_commit_pair(&qk_done[slot_of(jq, k >> 1)]);
               }
-              rope_pending = true;
+              mma_commit_pair(&qk_done[s]);
+              ++qk_k;
               prog = true;
+            }
+            if (qk_k == 4) {
+              rope_pending = true;
+              qk_k = 0;
             }
           }
           if (rope_pending && mbar_test(smem_u32(rope_full), jq & 1)) {
@@ -422,6 +490,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     };
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    const int tunit_sm = rank == 0 ? worker : 256 + worker;  // trace slot of this CTA's softmax
+    (void)tunit_sm;
     TileCursor c;
     c.init(a, range);
     while (ok && !c.done()) {
@@ -434,7 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         ok = false;
         break;
       }
-      if (L == 0) MLA_TRACE_EVENT(tunit, 8, j);
+      if (L == 0) MLA_TRACE_EVENT(tunit_sm, 8, j);
       tc_fence_after();
       float s[64];
 #pragma unroll
@@ -460,7 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         if (rank == 0)
           mbar_arrive(&s_free[j & 1]);
         else
-          mbar_arrive_cluster(l_sfree[j & 1]);
+          PAIR_ARRIVE(l_sfree[j & 1]);
       }
       const float m_new = fmaxf(m_run, fmaxf(pmax, rb[L ^ 64]));
       if (j >= 1) {
@@ -469,7 +539,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           ok = false;
           break;
         }
-        if (L == 0) MLA_TRACE_EVENT(tunit, 9, j - 1);
+        if (L == 0) MLA_TRACE_EVENT(tunit_sm, 9, j - 1);
         tc_fence_after();
       }
       const bool grow = __any_sync(0xffffffffu, m_new > m_run + ATT_RESCALE_LOG2);
@@ -513,8 +583,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         if (rank == 0)
           mbar_arrive(p_full);
         else
-          mbar_arrive_cluster(l_pfull);
-        MLA_TRACE_EVENT(tunit, 10, j);
+          PAIR_ARRIVE(l_pfull);
+        MLA_TRACE_EVENT(tunit_sm, 10, j);
       }
       if (c.last()) {
         // ---------------------------------------------------------- epilogue of the segment

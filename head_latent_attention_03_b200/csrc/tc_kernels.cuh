@@ -622,15 +622,14 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   a.lse_part = aw.lse_part;
   cudaError_t e;
   if (pair) {
-    CUtensorMap m1, m2, m8;
+    CUtensorMap m1, m2;
     if (!map_cache_chunks(&m1, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 1) ||
-        !map_cache_chunks(&m2, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 2) ||
-        !map_cache_chunks(&m8, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 8))
+        !map_cache_chunks(&m2, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 2))
       return MLA_ERR_CUDA;
     dim3 grid(2 * p.workers);
     cudaFuncSetAttribute(mla_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
     // cluster dimensions are compiled in (__cluster_dims__)
-    e = launch_pdl(mla_attn_pair_kernel, grid, dim3(PairCfg::THREADS), PairCfg::SMEM, st, 1, mq, mr, m1, m2, m8, a);
+    e = launch_pdl(mla_attn_pair_kernel, grid, dim3(PairCfg::THREADS), PairCfg::SMEM, st, 1, mq, mr, m1, m2, a);
   } else {
     dim3 grid(p.workers * attn_groups(D));
     e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
