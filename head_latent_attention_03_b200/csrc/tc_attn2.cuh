@@ -533,6 +533,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           PAIR_ARRIVE(l_sfree[j & 1]);
       }
       const float m_new = fmaxf(m_run, fmaxf(pmax, rb[L ^ 64]));
+      // Warps q and q+2 hold the two page halves of the same 32 heads with
+      // equal (m_new, m_run), so both take the same decision.
+      const bool grow = __any_sync(0xffffffffu, m_new > m_run + ATT_RESCALE_LOG2);
+      float alpha = 1.f;
+      bool rescale = false;
+      if (c.first()) {
+        m_run = m_new;  // PV of a segment's first tile overwrites O
+      } else if (grow) {
+        alpha = exp2_approx(m_run - m_new);
+        l_run *= alpha;
+        m_run = m_new;
+        rescale = true;
+      }
+      // P of this tile in registers first: only its store into the P buffer
+      // (still read by PV(j-1)) and a rescale of O wait for PV(j-1)
+      uint32_t pk[8][4];
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = exp2_approx(s[8 * cc + 2 * e] - m_run);
+          const float p1 = exp2_approx(s[8 * cc + 2 * e + 1] - m_run);
+          l_run += p0 + p1;
+          pk[cc][e] = pack_bf16(p0, p1);
+        }
+      }
       if (j >= 1) {
         // PV(j-1) complete: the P buffer is free and O is stable
         if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 523)) {
@@ -542,13 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         if (L == 0) MLA_TRACE_EVENT(tunit_sm, 9, j - 1);
         tc_fence_after();
       }
-      const bool grow = __any_sync(0xffffffffu, m_new > m_run + ATT_RESCALE_LOG2);
-      if (c.first()) {
-        m_run = m_new;  // PV of a segment's first tile overwrites O
-      } else if (grow) {
-        const float alpha = exp2_approx(m_run - m_new);
-        l_run *= alpha;
-        m_run = m_new;
+      if (rescale) {
 #pragma unroll 1
         for (int cc = 0; cc < 256; cc += 16) {
           float o[16];
@@ -562,17 +582,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       }
       uint8_t* prow = smem + C::OFF_P + g * 8192 + h * 128;
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = exp2_approx(s[8 * cc + 2 * e] - m_run);
-          const float p1 = exp2_approx(s[8 * cc + 2 * e + 1] - m_run);
-          l_run += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
-        }
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) << 4)) = make_uint4(pk[cc][0], pk[cc][1], pk[cc][2], pk[cc][3]);
       fence_proxy_async_smem();
       tc_fence_before();
       if (!group_sync(526)) {
