@@ -61,8 +61,12 @@ namespace mla {
 #define PAIR_TEST(a, p) mbar_test(a, p)
 #endif
 
+#ifndef PAIR_BACKOFF_NS
+#define PAIR_BACKOFF_NS 32  // MMA issuer's back-off between fruitless polls
+#endif
+
 #ifndef PAIR_PREFETCH
-#define PAIR_PREFETCH 1  // tiles of own pages prefetched into L2 ahead of their load
+#define PAIR_PREFETCH 1  // own pages are prefetched into L2 this many tiles ahead of their load (>= 1)
 #endif
 
 struct PairCfg {
@@ -217,9 +221,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       tma_prefetch_desc(&m_page2);
       const uint32_t lq = mapa_shared(smem_u32(q_full), 0);
       const uint32_t l_rope = mapa_shared(smem_u32(rope_full), 0);
-      // Own pages are prefetched into L2 PAIR_PREFETCH tiles ahead: the TMA
-      // loads below, and the other CTA's refills from this page, then see L2
-      // rather than HBM latency, which no shared-memory ring could cover.
+      // Own pages are prefetched into L2 PAIR_PREFETCH tiles ahead (one tile
+      // measured best): the loads below, and the other CTA's refills from
+      // this page, then see L2 rather than HBM latency.
       constexpr uint32_t PAGE_BYTES = 64u * (ATT_DC + ATT_DR) * 2u;
       TileCursor c, cf;
       c.init(a, range);
@@ -233,7 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
       };
       if (!cf.done()) cf.step(a);
-      for (int i = 0; i < PAIR_PREFETCH; ++i) prefetch();
+      for (int i = 1; i < PAIR_PREFETCH; ++i) prefetch();
       while (!c.done()) {
         const int g = c.g;
         // the RoPE slot, and at a segment's start the Q buffer, are free once
@@ -458,7 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           t_idle = 0;
           spins = 0;
         } else if ((++spins & 63u) != 0) {
-          __nanosleep(32);
+          if (PAIR_BACKOFF_NS > 0) __nanosleep(PAIR_BACKOFF_NS);
         } else {
           if (*abort_flag) break;
           const uint64_t now = globaltimer_ns();
