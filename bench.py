@@ -317,7 +317,10 @@ def run_ours(args):
         else:
             roof = {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": tensor, "unit": "TFLOP/s",
                     "frac": round(achieved_tf / tensor, 4)}
-        roof.update({"traffic": traffic, "kernel": "mla_attn_kernel (+ mla_combine_kernel)",
+        attn_kernel = "mla_attn_pair_kernel" if w.dims.n_h == 128 else "mla_attn_kernel"
+        roof.update({"traffic": traffic,
+                     "kernel": f"attention stage timed as one: mla_attn_plan_kernel + {attn_kernel} + mla_combine_kernel"
+                               f" (traffic: {attn_kernel} alone)",
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
                      "other_roof": {"hbm_frac": round(achieved_gbs / hbm, 4),
                                     "tensor_frac": round(achieved_tf / tensor, 4),
