@@ -61,6 +61,9 @@ namespace mla {
 #define PAIR_TEST(a, p) mbar_test(a, p)
 #endif
 
+#ifndef PAIR_WARP_ARRIVE
+#define PAIR_WARP_ARRIVE 1  // P written: one arrive per softmax warp instead of a group barrier
+#endif
 #ifndef PAIR_BACKOFF_NS
 #define PAIR_BACKOFF_NS 32  // MMA issuer's back-off between fruitless polls
 #endif
@@ -150,7 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       mbar_init(&pv_done[i], 1);
       mbar_init(&z_land[i], 1);
     }
-    mbar_init(p_full, 2);
+    mbar_init(p_full, PAIR_WARP_ARRIVE ? 8 : 2);
     mbar_init(last_ready, 2);
     mbar_init(grp_bar, 128);
     *abort_flag = 0;
@@ -590,6 +593,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) << 4)) = make_uint4(pk[cc][0], pk[cc][1], pk[cc][2], pk[cc][3]);
       fence_proxy_async_smem();
       tc_fence_before();
+#if PAIR_WARP_ARRIVE
+      // each warp announces its own stores (p_full counts 4 warps x 2 CTAs)
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(p_full);
+        else
+          PAIR_ARRIVE(l_pfull);
+        if (L == 0) MLA_TRACE_EVENT(tunit_sm, 10, j);
+      }
+#else
       if (!group_sync(526)) {
         ok = false;
         break;
@@ -601,6 +615,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           PAIR_ARRIVE(l_pfull);
         MLA_TRACE_EVENT(tunit_sm, 10, j);
       }
+#endif
       if (c.last()) {
         // ---------------------------------------------------------- epilogue of the segment
         // O is read out before this thread writes the next segment's first P,

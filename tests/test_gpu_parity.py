@@ -169,6 +169,15 @@ def test_bad_page_id_reports_capacity_error():
 # full-size workloads, in the launch configuration bench.py times; the oracle
 # checks a sample of sequences
 # ----------------------------------------------------------------------------
+def test_plan_over_many_rows():
+    # More decode rows than the plan kernel's 1024 threads: its scans run in
+    # two chunks whose carries decide every later row's segments and slots.
+    # Short ragged caches cut most rows across CTAs (combine on).  Rows on
+    # both sides of the chunk boundary are checked.
+    w = dataclasses.replace(I.WORKLOADS["lite"], name="lite_many", batch=1100, prior="uniform:0:200")
+    check_decode(w, seqs=[0, 1, 511, 1022, 1023, 1024, 1025, 1099])
+
+
 @pytest.mark.parametrize("name,seqs", [("lite", [0, 31]), ("v2", None)])
 def test_full_size_sampled(name, seqs):
     w = I.WORKLOADS[name]
