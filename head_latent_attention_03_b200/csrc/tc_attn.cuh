@@ -5,18 +5,25 @@
 //   s_j = scale * (q_lat_i . c^KV_j + q^R_i . k^R_j),   o_lat_i = sum_j softmax(s)_j c^KV_j
 // over the shared paged cache rows [c^KV_j | k^R_j] (d_c = 512, d_h^R = 64).
 //
-// Work unit: (query row r, group of H heads, KV split).  Both contractions run
-// as tcgen05 MMAs with the cached tokens on M = 128 ("swap-AB"): the group's
-// H heads are the N dimension, so one 128-token cache tile feeds
+// This file holds the attention work plan (mla_attn_plan_kernel: rows cut
+// into segments of 128-token tiles, dealt to CTAs), the one-CTA attention
+// kernel for layers of up to 64 heads, and the LSE combine; 128-head layers
+// use the CTA-pair kernel of tc_attn2.cuh on the same plan.
+//
+// One-CTA kernel.  A CTA = one group of H heads walking its list of segments
+// (query row, token range).  Both contractions run as tcgen05 MMAs with the
+// cached tokens on M = 128 ("swap-AB"): the group's H heads are the N
+// dimension, so one 128-token cache tile feeds
 //   S^T[128 tok x H]   = Kt[128 x 576]   . Q^T      (A = tile, K-major)
 //   O^T[512 x H]      += V^T[512 x 128] . P^T      (A = same tile, MN-major)
-// The 576-wide cache row is read from HBM once per unit and used by both
+// The 576-wide cache row is read from HBM once per CTA and used by both
 // products straight from shared memory.  S^T and O^T live in TMEM
 // (2*H + 4*H fp32 columns).
 //
 // Roles (192 threads):
-//   warp 0      TMA producer: Q once, then per tile one 16 KB RoPE slot and
-//               four 32 KB latent slots (2 pages x 128 latent columns)
+//   warp 0      TMA producer: Q once per segment, then per tile one 16 KB
+//               RoPE slot and four 32 KB latent slots (2 pages x 128 latent
+//               columns)
 //   warp 1      MMA issuer (one thread) and TMEM owner; QK(j+1) runs while
 //               the softmax of tile j does, PV(j) as soon as P(j) is written
 //   warps 2..5  softmax: thread = token row of the tile.  Tile max per head by

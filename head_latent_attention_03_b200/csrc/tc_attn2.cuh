@@ -36,9 +36,10 @@
 //   6    other-page producer: refills the pair slots PV needs once QK is done
 //        with them; zeroes rows past kv_len in the last tile
 // TMA pair loads complete their bytes on the leader's barriers, for which the
-// leader alone posts the byte count; the only cluster-scope arrives are one
-// per CTA per tile from the softmax (S consumed, P written) and the last
-// tile's zeroing.  All waits are bounded.
+// leader alone posts the byte count; the other CTA's only arrives on the
+// leader's barriers are "S read" (one per tile), "P written" (one per softmax
+// warp and tile) and the last tile's zeroing, all with CTA-scope release.
+// All waits are bounded.
 #pragma once
 
 #include "common.cuh"

@@ -1,8 +1,10 @@
 // tc_kernels.cuh — host side of the bf16 tensor-core path.
 //
-// Builds TMA descriptors over the caller's buffers, plans K splits and KV
-// splits from the SM count, carves the caller's workspace and launches the
-// GEMM / attention / finishing kernels on the caller's stream.
+// Builds TMA descriptors over the caller's buffers, plans the projections'
+// K splits (thread-block clusters) and the attention's work plan from the SM
+// count, carves the caller's workspace and launches the GEMM, plan, attention
+// and combine kernels on the caller's stream with programmatic dependent
+// launch.
 #pragma once
 
 #include <cuda.h>

@@ -34,6 +34,11 @@
  *  - There is no CPU fallback and no dispatch to other devices: a shape the
  *    kernels do not support returns MLA_ERR_UNSUPPORTED.
  *  - Results are deterministic for fixed arguments (no atomics in reductions).
+ *  - bf16 kernels launch with programmatic stream serialisation: each may
+ *    start (set-up, L2 prefetch of weights) while the previous kernel on the
+ *    stream is finishing, but reads no buffer and writes nothing before that
+ *    kernel has completed, so any stream-ordered producer of an argument —
+ *    weights included — is safe.
  *
  * Supported shapes.
  *  MLA_F32 (exact fp32 SIMT kernels): d_hr even, block_size >= 1, any d, n_h,
