@@ -157,9 +157,6 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ---------------------------------------------------------------------------
 // TMA tiled loads into the issuing CTA's shared memory
@@ -343,40 +340,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cl_addr) {
   asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
 }
-__device__ __forceinline__ void mbar_expect_tx_cluster(uint32_t cl_addr, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cl_addr),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// bounded wait with cluster-scope acquire (barriers that receive remote arrivals)
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
-  const uint32_t addr = smem_u32(bar);
-  if (mbar_try_wait_cluster(addr, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  const uint64_t limit = g_spin_limit_ns;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait_cluster(addr, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (abort && *abort) return false;
-      if (globaltimer_ns() - t0 > limit) {
-        record_error(ERR_TIMEOUT, site);
-        if (abort) *abort = 1;
-        return false;
-      }
-    }
-  }
-}
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start while the previous kernel of the stream is still
 // running; pdl_wait() blocks until that kernel has completed and its memory
@@ -394,16 +357,8 @@ __device__ __forceinline__ float2 ld_cluster_f2(uint32_t addr) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// TMA tile load into this CTA's shared memory that completes bytes on the
+// TMA tile loads into this CTA's shared memory that complete bytes on the
 // mbarrier at shared::cluster address `cl_bar` (the pair's leader CTA).
-__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t cl_bar, int x, int y,
-                                                 int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(cl_bar), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t cl_bar, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"

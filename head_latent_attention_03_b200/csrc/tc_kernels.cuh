@@ -263,8 +263,6 @@ inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan
   return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-inline unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
-
 inline RopeParams rope_of(const mla_layer_desc* D) {
   RopeParams r;
   r.base = D->rope_base;
