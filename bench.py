@@ -184,6 +184,17 @@ def cpu_oracle_baseline(w, seconds: float = 12.0):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings over the process group (the
+    slowest rank times the job); the values themselves without one."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -263,10 +274,7 @@ def run_ours(args):
         raise RuntimeError(f"device status after timed steps: {mla.status_string(code)}")
     t_ms = e0.elapsed_time(e1)
     attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
-    t_all = torch.tensor([t_ms, attn_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
-    t_ms, attn_ms = float(t_all[0]), float(t_all[1])
+    t_ms, attn_ms = max_over_ranks([t_ms, attn_ms], dev)
 
     # end to end through the public API: pinned host inputs in, result out, every step
     h_host = st.h.cpu().pin_memory()
@@ -297,9 +305,8 @@ def run_ours(args):
         e2e_step()
     f1.record(stream)
     torch.cuda.synchronize()
-    t_e2e = torch.tensor([max(f0.elapsed_time(f1), 1e-9)], dtype=torch.float64, device=dev)
+    (t_e2e,) = max_over_ranks([max(f0.elapsed_time(f1), 1e-9)], dev)
     if world > 1:
-        dist.all_reduce(t_e2e, op=dist.ReduceOp.MAX)
         dist.barrier()
 
     if rank == 0:
@@ -327,7 +334,7 @@ def run_ours(args):
                                     "attn_bytes_per_launch": attn_bytes, "attn_flops_per_launch": attn_flops,
                                     "attn_us": round(attn_ms * 1e3, 2)}})
         value = world * rows * args.steps / (t_ms * 1e-3)
-        e2e_value = world * rows * e2e_steps / (float(t_e2e[0]) * 1e-3) if e2e_steps else None
+        e2e_value = world * rows * e2e_steps / (t_e2e * 1e-3) if e2e_steps else None
         out = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(t_ms / args.steps, 4),
