@@ -118,6 +118,15 @@ def test_bf16_small(w):
     check_decode(w)
 
 
+@pytest.mark.parametrize("n_h,splits", [(32, 0), (32, 3), (64, 0), (64, 3)])
+def test_bf16_other_head_counts(n_h, splits):
+    # 32 and 64 heads: the one-CTA kernel with one or two 32-head groups per
+    # row (the groups of a segment run side by side), automatic and explicit
+    # splits.
+    w = dataclasses.replace(LITE_SMALL, name=f"heads{n_h}", dims=dataclasses.replace(I.LITE, n_h=n_h))
+    check_decode(w, num_splits=splits)
+
+
 @pytest.mark.parametrize("splits", [1, 2, 5])
 def test_split_count_invariance(splits):
     w = dataclasses.replace(LITE_SMALL, prior="list:300,1500,900,64")
