@@ -56,3 +56,23 @@ def test_invalid_arguments_are_rejected_without_a_gpu(lib):
     bad = mla.layer_desc(V2)
     bad.d_hr = 63  # odd RoPE width
     assert mla.workspace_size(bad, 1, 1, 64) == 0
+
+
+def declared_arity():
+    """Number of parameters of every function include/mla.h declares."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(mla_[a-z_]+)\s*\(([^)]*)\)\s*;", src):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_marshals_every_declared_entry_point_with_its_arity():
+    # the ctypes signatures in mla.py are the only marshalling layer: every
+    # declared function must be bound, with exactly the header's parameters
+    arity = declared_arity()
+    assert set(arity) - set(mla._SIGS) == set(), set(arity) - set(mla._SIGS)
+    for name, (_, argtypes) in mla._SIGS.items():
+        assert name in arity, name
+        assert len(argtypes) == arity[name], (name, len(argtypes), arity[name])
