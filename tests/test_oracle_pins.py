@@ -303,3 +303,21 @@ def test_self_score_is_unrotated_dot():
     scale = D.attn_logit_factor / math.sqrt(D.d_h + D.d_hr)
     ref = np.log(L + np.exp(scale * (qr @ kr)))
     assert np.max(np.abs(res["lse"] - ref)) < 1e-12
+
+
+# Paged cache ([explainer] 2.2.2: one cached row [c^KV | k^R] per token, here
+# in 64-token pages reached through a page table).  The generator draws each
+# sequence's prior rows in token order from its own seeded stream before
+# scattering them over permuted pages; the oracle's gather must return exactly
+# that order (a swapped page/slot index or a shifted slot reads other rows).
+def test_gather_rows_returns_rows_in_token_order():
+    import dataclasses
+    from head_latent_attention_03_b200 import inputs as I
+    D = dataclasses.replace(TINY, block_size=8)
+    w = I.Workload("gather_pin", 7, D, 3, "list:5,17,30", permute_pages=True)
+    batch = I.gen_batch(w)
+    assert not np.array_equal(batch.block_table[:, 0], np.arange(3))  # pages really permuted
+    for b, L in enumerate(batch.prior_len):
+        want = I._store(I._normal(I.rng_for(w.cfg_id, I._T_PRIOR, b), (int(L), D.row), 1.0), D)
+        got = O.gather_rows(batch.pool, batch.block_table[b], int(L), D.block_size)
+        assert np.array_equal(got, want.astype(np.float64)), b

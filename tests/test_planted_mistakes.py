@@ -38,6 +38,9 @@ MUTATIONS = {
     # YaRN blend with the wrong end points
     "yarn_blend_swapped": ("out[i] = (1.0 - g) * theta[i] / yarn_scale + g * theta[i]",
                            "out[i] = g * theta[i] / yarn_scale + (1.0 - g) * theta[i]"),
+    # paged-cache gather reading the neighbouring slot of each page
+    "gather_slot_shift": ("out[j] = pool[table_row[j // block], j % block]",
+                          "out[j] = pool[table_row[j // block], (j + 1) % block]"),
     # W^O applied before W^UV's head split is undone
     "out_proj_heads": ("o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64))",
                        "o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64)[::-1])"),
