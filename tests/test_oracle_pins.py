@@ -321,3 +321,23 @@ def test_gather_rows_returns_rows_in_token_order():
         want = I._store(I._normal(I.rng_for(w.cfg_id, I._T_PRIOR, b), (int(L), D.row), 1.0), D)
         got = O.gather_rows(batch.pool, batch.block_table[b], int(L), D.block_size)
         assert np.array_equal(got, want.astype(np.float64)), b
+
+
+# Data flow of the decoupled RoPE parts ([explainer] 2.2.2): the shared key
+# k^R is computed from h_t itself, not from the latent c^KV, and both query
+# parts come from the query latent c^Q.  Zeroing W^DKV must leave k^R intact;
+# zeroing W^DQ must silence q^C and q^R.
+def test_key_rope_comes_from_h_and_query_parts_from_the_query_latent():
+    D = SMALL[1]  # query compression on (d_cq > 0)
+    rng = np.random.default_rng(11)
+    W = _rand_weights(D, rng)
+    h = rng.standard_normal(D.d)
+    W0 = dict(W, w_dkv=np.zeros_like(W["w_dkv"]))
+    row = O.compress_kv(D, W0, h, 5)
+    assert np.all(row[:D.d_c] == 0)
+    assert np.linalg.norm(row[D.d_c:]) > 0.1 * np.linalg.norm(O.compress_kv(D, W, h, 5)[D.d_c:])
+    W1 = dict(W, w_dq=np.zeros_like(W["w_dq"]))
+    q_c, q_r = O.queries(D, W1, h, 5)
+    assert np.all(q_c == 0) and np.all(q_r == 0)
+    q_c, q_r = O.queries(D, W, h, 5)
+    assert np.linalg.norm(q_c) > 0 and np.linalg.norm(q_r) > 0
