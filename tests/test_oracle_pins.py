@@ -341,3 +341,23 @@ def test_key_rope_comes_from_h_and_query_parts_from_the_query_latent():
     assert np.all(q_c == 0) and np.all(q_r == 0)
     q_c, q_r = O.queries(D, W, h, 5)
     assert np.linalg.norm(q_c) > 0 and np.linalg.norm(q_r) > 0
+
+
+# Vanishing queries (eq 7 with every logit zero): the softmax is uniform over
+# the L + 1 visible rows (prior rows and the new token), so each head's o_lat
+# is the plain mean of their c^KV parts, the new row included, and the lse is
+# log(L + 1).
+def test_vanishing_queries_attend_uniformly_over_all_visible_rows():
+    for D in SMALL:
+        rng = np.random.default_rng(13)
+        W = _rand_weights(D, rng)
+        W = dict(W, w_uq=np.zeros_like(W["w_uq"]), w_qr=np.zeros_like(W["w_qr"]))
+        L = 9
+        prior = rng.standard_normal((L, D.d_c + D.d_hr))
+        h = rng.standard_normal(D.d)
+        out = O.decode_token(D, W, h, L, prior, absorbed=True)
+        rows = np.concatenate([prior, out["row"][None, :]], axis=0)
+        want = rows[:, :D.d_c].mean(axis=0)
+        for i in range(D.n_h):
+            np.testing.assert_allclose(out["o_lat"][i], want, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(out["lse"], math.log(L + 1), rtol=1e-12)
