@@ -94,7 +94,7 @@ def test_mha_equivalence_stacked_factorisation():
 
 
 def test_mha_equivalence_padded_latent():
-    # d_c > d: W^DKV = [I; 0], W^UK = [W^K, 0] (the benchmark spec's d_c >= n_h d_h case).
+    # d_c > d: W^DKV = [I; 0], W^UK = [W^K, 0] (the case d_c >= n_h d_h).
     n_h, d_h, d, d_c = 2, 8, 16, 24
     D = LayerDims(d=d, n_h=n_h, d_h=d_h, d_c=d_c, d_cq=0, d_hr=0, dtype="f32")
     rng = np.random.default_rng(5)
