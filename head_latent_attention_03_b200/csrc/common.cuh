@@ -60,7 +60,7 @@ __device__ __forceinline__ bool elect_one() {
 // mla_trace_read().  Compiles to nothing otherwise.
 // ---------------------------------------------------------------------------
 #ifdef MLA_TRACE
-constexpr int MLA_TRACE_UNITS = 512, MLA_TRACE_EVENTS = 16, MLA_TRACE_TILES = 40;
+constexpr int MLA_TRACE_UNITS = 512, MLA_TRACE_EVENTS = 28, MLA_TRACE_TILES = 40;
 __device__ unsigned long long g_trace[MLA_TRACE_UNITS][MLA_TRACE_EVENTS][MLA_TRACE_TILES];
 __device__ __forceinline__ void trace_event(int unit, int ev, int tile) {
   if (unit >= 0 && unit < MLA_TRACE_UNITS && tile >= 0 && tile < MLA_TRACE_TILES)
@@ -134,6 +134,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(addr, parity)) return true;
     if ((it & 63u) == 0) {
+      if (abort && *abort) return false;
+      if (globaltimer_ns() - t0 > limit) {
+        record_error(ERR_TIMEOUT, site);
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// mbar_wait for latency-critical waits: polls with test_wait (never
+// suspends the thread), with the same time limit and abort handling.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
+  const uint32_t addr = smem_u32(bar);
+  if (mbar_test(addr, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = g_spin_limit_ns;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(addr, parity)) return true;
+    if ((it & 255u) == 0) {
       if (abort && *abort) return false;
       if (globaltimer_ns() - t0 > limit) {
         record_error(ERR_TIMEOUT, site);
@@ -392,6 +412,19 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, 
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D (+)= A * B^T across the CTA pair with A read from tensor memory.  For
+// M = 128 each CTA holds its 64 rows of A twice, in lanes r and 64 + r (both
+// halves of the data path read their own lanes), K packed two bf16 values per
+// 32-bit column, even element in the low half.
+__device__ __forceinline__ void mma_bf16_pair_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive on the mbarrier at the same offset in both CTAs of the pair once all

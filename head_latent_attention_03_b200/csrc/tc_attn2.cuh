@@ -13,6 +13,13 @@
 // columns and O 256: the fp32 O of all 128 heads (256 KB) no longer has to fit
 // one SM.  Q of 64 heads (72 KB) stays resident in shared memory.
 //
+// P lives in TMEM as the A operand of PV (two buffers, by tile parity), so
+// the softmax of tile j+1 never waits for PV(j).  A 2-SM M = 128 MMA reads A
+// from both lane halves of each CTA (lanes r and 64 + r hold row r with the
+// instruction's whole K), while a softmax thread computes one page of its
+// head; the two threads of a head swap halves through a 16 KB shared-memory
+// staging buffer and both store all 128 tokens.
+//
 // Cache data flow.  Each CTA loads its own page's row once, as a RoPE chunk
 // and four latent "pairs" (chunks 2k, 2k+1: 16 KB), and QK reads them.  PV
 // instruction (i, p) — latent columns of instruction i, tokens of page p —
@@ -30,7 +37,8 @@
 // 2-chunk own-page boxes, plus two 2-chunk refill boxes.
 //
 // Warps (224 threads per CTA):
-//   0    own-page producer (RoPE chunk + four latent pairs per tile)
+//   0    own-page producer (four latent pairs per tile as their slots free
+//        up, then the RoPE chunk once QK of the previous tile is done)
 //   1    MMA issuer (leader CTA only, one thread) and TMEM owner (both CTAs)
 //   2-5  softmax: thread = (head, page half of the tile)
 //   6    other-page producer: refills the pair slots PV needs once QK is done
@@ -69,19 +77,32 @@ namespace mla {
 #define PAIR_BACKOFF_NS 32  // MMA issuer's back-off between fruitless polls
 #endif
 
+#ifndef PAIR_SM_SPIN
+#define PAIR_SM_SPIN 0  // 1: the softmax warps poll their barriers without suspending
+#endif
+#if PAIR_SM_SPIN
+#define PAIR_SM_WAIT mbar_wait_spin
+#else
+#define PAIR_SM_WAIT mbar_wait
+#endif
+
+#ifndef PAIR_QK_CUTIN
+#define PAIR_QK_CUTIN 0  // 1: the MMA issuer re-checks PV between the latent pairs of a QK
+#endif
+
 #ifndef PAIR_PREFETCH
 #define PAIR_PREFETCH 1  // own pages are prefetched into L2 this many tiles ahead of their load (>= 1)
 #endif
 
 struct PairCfg {
-#ifdef MLA_TRACE
+#if defined(MLA_TRACE) && defined(MLA_TRACE_OBSERVER)
   static constexpr int THREADS = 256;  // + a barrier-observer warp
 #else
   static constexpr int THREADS = 224;
 #endif
   static constexpr int Q_CHUNK = 64 * 128;        // 64 heads x 64 columns
   static constexpr int Q_BYTES = 9 * Q_CHUNK;     // 72 KB
-  static constexpr int P_BYTES = 2 * 64 * 128;    // 64 heads x 128 tokens (two SW128 K atoms)
+  static constexpr int P_BYTES = 2 * 64 * 128;    // staging: 64 heads x 2 pages x 64 tokens (bf16)
   static constexpr int PAIR = 16384;              // one page x 2 latent chunks
   static constexpr int ROPE = 8192;               // one page x 64 RoPE columns
   static constexpr int NP = 8;                    // pair slots (two tiles)
@@ -90,7 +111,7 @@ struct PairCfg {
   static constexpr int OFF_ROPE = OFF_P + P_BYTES;
   static constexpr int OFF_PAIR = OFF_ROPE + ROPE;
   static constexpr int OFF_BAR = OFF_PAIR + NP * PAIR;
-  static constexpr int N_BAR = 4 * NP + 1 + 1 + 2 + 2 + 1 + 2 + 1 + 1 + 2;
+  static constexpr int N_BAR = 4 * NP + 1 + 1 + 2 + 2 + 2 + 2 + 2 + 1 + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int OFF_RED = OFF_MISC + 16;
   static constexpr int SMEM = OFF_RED + 3 * 128 * 4 + 1024;
@@ -111,7 +132,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   // Pair commits per tile: one qk_done per pair slot (QK has read it: the
   // other CTA may refill it), one pv_slot per pair slot (PV has read it: the
   // next own-page load may overwrite it), s_full (S ready; the RoPE slot is
-  // free) and pv_done (O is stable, the P buffer is free).  s_full and
+  // free) and pv_done (O is stable, the tile's P buffer is free).  s_full and
   // pv_done have one instance per tile parity so that a waiter is never two
   // phases behind.
   uint64_t* own_full = bar;                   // leader [NP]: own-page pair landed in the slot
@@ -121,10 +142,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   uint64_t* q_full = rope_full + 1;           // leader
   uint64_t* s_full = q_full + 1;              // both [2]: pair commit after QK(j)
   uint64_t* s_free = s_full + 2;              // leader [2]: one arrive per CTA
-  uint64_t* p_full = s_free + 2;              // leader: one arrive per CTA
-  uint64_t* pv_done = p_full + 1;             // both [2]: pair commit after PV(j)
-  uint64_t* last_ready = pv_done + 2;         // leader: both CTAs zeroed the last tile
-  uint64_t* grp_bar = last_ready + 1;         // local: 128 softmax threads
+  uint64_t* p_full = s_free + 2;              // leader [2]: P(j) in TMEM, one arrive per softmax warp
+  uint64_t* pv_done = p_full + 2;             // both [2]: pair commit after PV(j)
+  uint64_t* last_ready = pv_done + 2;         // leader [2]: both CTAs zeroed the last tile
+  uint64_t* grp_bar = last_ready + 2;         // local: 128 softmax threads
   uint64_t* z_land = grp_bar + 1;             // local [2]: last tile's other-page refills
   uint64_t* pv_slot = z_land + 2;             // both [NP]: pair commit once PV has read the slot
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -154,8 +175,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       mbar_init(&pv_done[i], 1);
       mbar_init(&z_land[i], 1);
     }
-    mbar_init(p_full, PAIR_WARP_ARRIVE ? 8 : 2);
-    mbar_init(last_ready, 2);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], PAIR_WARP_ARRIVE ? 8 : 2);
+      mbar_init(&last_ready[i], 2);
+    }
     mbar_init(grp_bar, 128);
     *abort_flag = 0;
     fence_mbar_init();
@@ -173,6 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 0, 0);
   const uint32_t tS = tmem;         // S buffers: columns [0,64) and [64,128)
   const uint32_t tO = tmem + 128;   // O: columns [128,256) (d_c 0..255) and [256,384) (256..511)
+  const uint32_t tP = tmem + 384;   // P buffers (bf16, A operand of PV): columns [384,448) and [448,512)
 
   // cache block of page `page` of the cursor's row; past the row: num_blocks
   // (out of range: TMA reads zeros)
@@ -194,24 +218,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   // The CTA whose own page is k & 1 keeps its own columns there; the other CTA
   // refills the slot with columns 2*(2*(k>>1) + rank) .. +1 of page k & 1.
 
-#ifdef MLA_TRACE
+#if defined(MLA_TRACE) && defined(MLA_TRACE_OBSERVER)
   if (warp == 7) {
     if (lane != 0 || rank != 0) {
     } else {
-    // trace-only observer: completion times of each tile's first own pair,
-    // first refill and P (leader barriers), polled without blocking anyone
+    // trace-only observer: completion times of each tile's first and last
+    // own pair, first refill, S, P and PV (leader barriers), polled for two
+    // tiles at a time without blocking anyone
     TileCursor c;
     c.init(a, range);
-    while (!c.done() && !*abort_flag) {
-      const int g = c.g, s0 = slot_of(g, 0), u0 = use_of(g, 0);
-      const uint64_t t_start = globaltimer_ns();
-      bool seen_own = false, seen_oth = c.zero(), seen_p = false;
-      while (!(seen_own && seen_oth && seen_p) && globaltimer_ns() - t_start < 2000000ull && !*abort_flag) {
-        if (!seen_own && mbar_test(smem_u32(&own_full[s0]), u0 & 1)) { seen_own = true; MLA_TRACE_EVENT(tunit, 3, g); }
-        if (!seen_oth && mbar_test(smem_u32(&oth_full[s0]), u0 & 1)) { seen_oth = true; MLA_TRACE_EVENT(tunit, 4, g); }
-        if (!seen_p && mbar_test_cluster(smem_u32(p_full), g & 1)) { seen_p = true; MLA_TRACE_EVENT(tunit, 15, g); }
+    TileCursor c2 = c;
+    if (!c2.done()) c2.step(a);
+    uint32_t seen[2] = {0, 0};
+    const uint64_t t_start = globaltimer_ns();
+    while (!c.done() && !*abort_flag && globaltimer_ns() - t_start < 20000000ull) {
+      for (int w = 0; w < 2; ++w) {
+        const TileCursor& cc = w == 0 ? c : c2;
+        if (cc.done()) continue;
+        const int g = cc.g;
+        const int s0 = slot_of(g, 0), u0 = use_of(g, 0), s3 = slot_of(g, 3), u3 = use_of(g, 3);
+        uint32_t& m = seen[w];
+        if (cc.zero()) m |= 2u;
+        if (!(m & 1u) && mbar_test(smem_u32(&own_full[s0]), u0 & 1)) { m |= 1u; MLA_TRACE_EVENT(tunit, 3, g); }
+        if (!(m & 2u) && mbar_test(smem_u32(&oth_full[s0]), u0 & 1)) { m |= 2u; MLA_TRACE_EVENT(tunit, 4, g); }
+        if (!(m & 4u) && mbar_test_cluster(smem_u32(&p_full[g & 1]), (g >> 1) & 1)) { m |= 4u; MLA_TRACE_EVENT(tunit, 15, g); }
+        if (!(m & 8u) && mbar_test(smem_u32(&own_full[s3]), u3 & 1)) { m |= 8u; MLA_TRACE_EVENT(tunit, 18, g); }
+        if (!(m & 16u) && mbar_test(smem_u32(&s_full[g & 1]), (g >> 1) & 1)) { m |= 16u; MLA_TRACE_EVENT(tunit, 16, g); }
+        if (!(m & 32u) && mbar_test(smem_u32(&pv_done[g & 1]), (g >> 1) & 1)) { m |= 32u; MLA_TRACE_EVENT(tunit, 17, g); }
       }
-      c.step(a);
+      if (seen[0] == 63u) {
+        c = c2;
+        seen[0] = seen[1];
+        seen[1] = 0;
+        if (!c2.done()) c2.step(a);
+      }
     }
     }
   } else
@@ -244,23 +284,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       for (int i = 1; i < PAIR_PREFETCH; ++i) prefetch();
       while (!c.done()) {
         const int g = c.g;
-        // the RoPE slot, and at a segment's start the Q buffer, are free once
-        // QK(g-1) is done
-        if (g >= 1 && !mbar_wait(&s_full[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, 503)) break;
-        if (c.first()) {
-          if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
-          const int qrow = c.S.r * a.n_h + head0;
-          for (int k = 0; k < 8; ++k)
-            tma_load_2d_pair(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, lq, k * 64, qrow);
-          tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
-        }
         prefetch();
         const int blk = page_block(c, c.tok() / 64 + (int)rank);
-        if (rank == 0) mbar_expect_tx(rope_full, 2 * C::ROPE);
-        tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, 8, blk);
-        MLA_TRACE_EVENT(tunit, 1, g);
         // the own page pair by pair, each into its slot as soon as PV(g-2)
-        // has read that slot: QK(g) starts on the first pair to land
+        // has read that slot: QK(g) starts on the first pair to land.  These
+        // loads wait for nothing else, so tile g streams in while QK(g-1)
+        // still runs.
         bool ok = true;
         for (int k = 0; k < 4 && ok; ++k) {
           const int s = slot_of(g, k), u = use_of(g, k);
@@ -271,9 +300,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           if (rank == 0) mbar_expect_tx(&own_full[s], 2 * C::PAIR);
           tma_load_4d_pair(smem + C::OFF_PAIR + s * C::PAIR, &m_page2, mapa_shared(smem_u32(&own_full[s]), 0), 0, 0,
                            2 * k, blk);
+          if (k == 0) MLA_TRACE_EVENT(tunit, 1, g);
+          if (k == 3) MLA_TRACE_EVENT(tunit, 2, g);
         }
         if (!ok) break;
-        MLA_TRACE_EVENT(tunit, 2, g);
+        // the RoPE slot, and at a segment's start the Q buffer, are free once
+        // QK(g-1) is done (QK reads the RoPE chunk last)
+        if (g >= 1 && !mbar_wait(&s_full[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, 503)) break;
+        if (c.first()) {
+          if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
+          const int qrow = c.S.r * a.n_h + head0;
+          for (int k = 0; k < 8; ++k)
+            tma_load_2d_pair(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, lq, k * 64, qrow);
+          tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
+        }
+        if (rank == 0) mbar_expect_tx(rope_full, 2 * C::ROPE);
+        tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, 8, blk);
+        MLA_TRACE_EVENT(tunit, 19, g);
         c.step(a);
       }
     }
@@ -335,7 +378,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && ok) PAIR_ARRIVE(mapa_shared(smem_u32(last_ready), 0));
+        if (lane == 0 && ok) PAIR_ARRIVE(mapa_shared(smem_u32(&last_ready[nz & 1]), 0));
         ++nz;
       }
       c.step(a);
@@ -348,7 +391,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       const uint32_t q_base = smem_u32(smem + C::OFF_Q);
       const uint32_t rope_base = smem_u32(smem + C::OFF_ROPE);
       const uint32_t pair0 = smem_u32(smem + C::OFF_PAIR);
-      const uint32_t p_base = smem_u32(smem + C::OFF_P);
       TileCursor cq, cp, cpost;  // next QK tile, next PV tile, PV tile + 2
       cq.init(a, range);
       cp = cq;
@@ -378,23 +420,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         // PV first: it frees the slots that later tiles' loads wait for
         if (cp.g < cq.g) {
           const int jp = cp.g;
-          if (!p_ok) p_ok = PAIR_TEST(smem_u32(p_full), jp & 1);
+          if (!p_ok) {
+            p_ok = PAIR_TEST(smem_u32(&p_full[jp & 1]), (jp >> 1) & 1);
+            if (p_ok) MLA_TRACE_EVENT(tunit, 15, jp);
+          }
           if (p_ok) {
             const bool zero = cp.zero();
             while (pv_k < 4) {
               const int s = slot_of(jp, pv_k), u = use_of(jp, pv_k);
-              const bool ready = zero ? PAIR_TEST(smem_u32(last_ready), nz & 1)
+              const bool ready = zero ? PAIR_TEST(smem_u32(&last_ready[nz & 1]), (nz >> 1) & 1)
                                       : mbar_test(smem_u32(&oth_full[s]), u & 1);
               if (!ready) break;
               if (pv_k == 0) MLA_TRACE_EVENT(tunit, 14, jp);
+              if (pv_k == 1) MLA_TRACE_EVENT(tunit, 20, jp);
+              if (pv_k == 2) MLA_TRACE_EVENT(tunit, 21, jp);
               tc_fence_after();
               const int i = pv_k >> 1, p = pv_k & 1;
               const uint32_t pb = pair0 + s * C::PAIR;
+              // P of page p, tokens 16kk..16kk+15: columns 32p + 8kk of the tile's P buffer
+              const uint32_t pa = tP + (jp & 1) * 64 + 32 * p;
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = smem_desc(p_base + p * 8192 + kk * 32, 16, 1024, SW128);
                 const uint64_t bd = smem_desc(pb + kk * 2048, 8192, 1024, SW128);
-                mma_bf16_pair(tO + 128 * i, ad, bd, id_pv, (cp.j > 0 || p > 0 || kk > 0) ? 1u : 0u);
+                mma_bf16_pair_ts(tO + 128 * i, pa + 8 * kk, bd, id_pv, (cp.j > 0 || p > 0 || kk > 0) ? 1u : 0u);
               }
               mma_commit_pair(&pv_slot[s]);
               // a zero tile's slots had no refill on oth_full: close that phase
@@ -440,6 +488,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
               mma_commit_pair(&qk_done[s]);
               ++qk_k;
               prog = true;
+              if (PAIR_QK_CUTIN && cp.g < cq.g) break;  // let PV of an older tile cut in
             }
             if (qk_k == 4) {
               rope_pending = true;
@@ -488,11 +537,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     const int g = L >> 6;            // which page of the tile this thread's scores cover
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t l_sfree[2] = {mapa_shared(smem_u32(&s_free[0]), 0), mapa_shared(smem_u32(&s_free[1]), 0)};
-    const uint32_t l_pfull = mapa_shared(smem_u32(p_full), 0);
+    const uint32_t l_pfull[2] = {mapa_shared(smem_u32(&p_full[0]), 0), mapa_shared(smem_u32(&p_full[1]), 0)};
     uint32_t gphase = 0;
     auto group_sync = [&](int site) -> bool {
       mbar_arrive(grp_bar);
-      const bool ok2 = mbar_wait(grp_bar, gphase & 1, abort_flag, site);
+      const bool ok2 = PAIR_SM_WAIT(grp_bar, gphase & 1, abort_flag, site);
       ++gphase;
       return ok2;
     };
@@ -508,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         m_run = -INFINITY;
         l_run = 0.f;
       }
-      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, 521)) {
+      if (!PAIR_SM_WAIT(&s_full[j & 1], (j >> 1) & 1, abort_flag, 521)) {
         ok = false;
         break;
       }
@@ -533,6 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         ok = false;
         break;
       }
+      if (L == 0) MLA_TRACE_EVENT(tunit_sm, 22, j);
       // every thread's TMEM reads of S(j) are complete: release the buffer
       if (L == 0) {
         if (rank == 0)
@@ -554,8 +604,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         m_run = m_new;
         rescale = true;
       }
-      // P of this tile in registers first: only its store into the P buffer
-      // (still read by PV(j-1)) and a rescale of O wait for PV(j-1)
+      // P of this tile in registers; its store into the tile's TMEM P buffer
+      // waits for PV(j-2), a rescale of O for PV(j-1)
       uint32_t pk[8][4];
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
@@ -567,13 +617,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           pk[cc][e] = pack_bf16(p0, p1);
         }
       }
-      if (j >= 1) {
-        // PV(j-1) complete: the P buffer is free and O is stable
-        if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, 523)) {
+      // Both TMEM lanes of a head (h and 64 + h) must hold P over all 128
+      // tokens of the tile (the duplicated A layout of the 2-SM MMA), but
+      // each thread computed one page: swap halves with the partner thread
+      // (same head, other page) through the staging buffer.  Its reuse by the
+      // next tile comes after that tile's max exchange, which every thread
+      // reaches only after reading this tile's halves.
+      uint4* stg = reinterpret_cast<uint4*>(smem + C::OFF_P);  // [page][8][64 heads]
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) stg[(g * 8 + cc) * 64 + h] = make_uint4(pk[cc][0], pk[cc][1], pk[cc][2], pk[cc][3]);
+      if (!group_sync(526)) {
+        ok = false;
+        break;
+      }
+      if (L == 0) MLA_TRACE_EVENT(tunit_sm, 23, j);
+      uint32_t po[8][4];
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const uint4 v = stg[((g ^ 1) * 8 + cc) * 64 + h];
+        po[cc][0] = v.x;
+        po[cc][1] = v.y;
+        po[cc][2] = v.z;
+        po[cc][3] = v.w;
+      }
+      // the P buffer of this tile was last read by PV(j-2); a rescale of O
+      // needs PV(j-1) complete
+      if (j >= 2 || (rescale && j >= 1)) {
+        const int jw = rescale ? j - 1 : j - 2;
+        if (!mbar_wait(&pv_done[jw & 1], (jw >> 1) & 1, abort_flag, 523)) {
           ok = false;
           break;
         }
-        if (L == 0) MLA_TRACE_EVENT(tunit_sm, 9, j - 1);
+        if (L == 0) MLA_TRACE_EVENT(tunit_sm, 9, j);
         tc_fence_after();
       }
       if (rescale) {
@@ -588,32 +663,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         }
         tmem_wait_st();
       }
-      uint8_t* prow = smem + C::OFF_P + g * 8192 + h * 128;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (h & 7)) << 4)) = make_uint4(pk[cc][0], pk[cc][1], pk[cc][2], pk[cc][3]);
-      fence_proxy_async_smem();
+      {
+        // columns [0,32): page 0's tokens, [32,64): page 1's; two tokens per column
+        const uint32_t pt = tP + (j & 1) * 64 + lane_off;
+        tmem_st32<32>(pt + 32 * g, reinterpret_cast<const float*>(&pk[0][0]));
+        tmem_st32<32>(pt + 32 * (g ^ 1), reinterpret_cast<const float*>(&po[0][0]));
+        tmem_wait_st();
+      }
       tc_fence_before();
 #if PAIR_WARP_ARRIVE
       // each warp announces its own stores (p_full counts 4 warps x 2 CTAs)
       __syncwarp();
       if (lane == 0) {
         if (rank == 0)
-          mbar_arrive(p_full);
+          mbar_arrive(&p_full[j & 1]);
         else
-          PAIR_ARRIVE(l_pfull);
+          PAIR_ARRIVE(l_pfull[j & 1]);
         if (L == 0) MLA_TRACE_EVENT(tunit_sm, 10, j);
+        if (L == 32) MLA_TRACE_EVENT(tunit_sm, 24, j);
+        if (L == 64) MLA_TRACE_EVENT(tunit_sm, 25, j);
+        if (L == 96) MLA_TRACE_EVENT(tunit_sm, 26, j);
       }
 #else
-      if (!group_sync(526)) {
+      if (!group_sync(528)) {
         ok = false;
         break;
       }
       if (L == 0) {
         if (rank == 0)
-          mbar_arrive(p_full);
+          mbar_arrive(&p_full[j & 1]);
         else
-          PAIR_ARRIVE(l_pfull);
+          PAIR_ARRIVE(l_pfull[j & 1]);
         MLA_TRACE_EVENT(tunit_sm, 10, j);
       }
 #endif
