@@ -227,14 +227,15 @@ mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* D, const void* q_lat,
   if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
   // The plan's unit list and partials must fit the array: an explicit split
   // count that does not fit is refused; the automatic plan deals the tiles
-  // out to fewer CTAs until it fits.
+  // out to the largest number of CTAs (CTA pairs) whose plan fits.
   const size_t cap = kNoAllocScratchBytes - 256;
   int workers = 0;
   if (num_splits > 0) {
     if (ws_attn(D, B, plan_attn(D, B, max_len, num_splits)) > cap) return MLA_ERR_CAPACITY;
   } else {
+    // the largest worker count whose plan fits (host arithmetic only)
     workers = attn_wave_workers(D);
-    while (workers > 1 && ws_attn(D, B, plan_attn(D, B, max_len, 0, workers)) > cap) workers /= 2;
+    while (workers > 1 && ws_attn(D, B, plan_attn(D, B, max_len, 0, workers)) > cap) --workers;
     if (ws_attn(D, B, plan_attn(D, B, max_len, 0, workers)) > cap) return MLA_ERR_CAPACITY;
   }
   return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, scratch, kNoAllocScratchBytes, num_splits,

@@ -725,35 +725,58 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
 // Merge the partials of rows cut into several units:
 // lse = log sum_s e^{lse_s}, o = sum_s e^{lse_s - lse} o_s.
-__global__ void mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                                   const int4* __restrict__ row_info, int n_h, __nv_bfloat16* __restrict__ o_lat,
-                                   float* __restrict__ lse) {
+// Block = (row, 8 heads, 1/CS of the latent columns), 256 threads; thread =
+// (head, 16/CS columns).  All loads of a part are independent and issued
+// together, so a thread pays the L2 latency about once per four parts; CS
+// > 1 spreads rows of few sequences (long contexts) over more blocks.
+constexpr int COMBINE_THREADS = 256, COMBINE_HEADS = 8;
+template <int CS>
+__global__ void __launch_bounds__(COMBINE_THREADS)
+    mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                       const int4* __restrict__ row_info, int n_h, __nv_bfloat16* __restrict__ o_lat,
+                       float* __restrict__ lse) {
+  constexpr int CPT = 16 / CS;  // columns per thread
   pdl_trigger();
   pdl_wait();
-  const int r = blockIdx.x / n_h, h = blockIdx.x % n_h;
+  const int groups = n_h / COMBINE_HEADS;
+  const int r = blockIdx.x / groups;
+  const int h = (blockIdx.x % groups) * COMBINE_HEADS + threadIdx.x / 32;
+  const int c0 = blockIdx.y * (ATT_DC / CS) + (threadIdx.x & 31) * CPT;
   const int4 info = row_info[r];
   const int n_parts = info.y, slot0 = info.z;
   if (n_parts <= 1) return;  // written directly by its unit
-  float mx = -INFINITY;
-  for (int s = 0; s < n_parts; ++s) mx = fmaxf(mx, lse_part[(long long)(slot0 + s) * n_h + h]);
-  float tot = 0.f;
-  for (int s = 0; s < n_parts; ++s) tot += expf(lse_part[(long long)(slot0 + s) * n_h + h] - mx);
-  const float lse_all = mx + logf(tot);
-  for (int d = threadIdx.x * 4; d < ATT_DC; d += blockDim.x * 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_parts; ++s) {
-      const float wgt = expf(lse_part[(long long)(slot0 + s) * n_h + h] - lse_all);
-      const float4 x = *reinterpret_cast<const float4*>(o_part + ((long long)(slot0 + s) * n_h + h) * ATT_DC + d);
-      acc.x += wgt * x.x;
-      acc.y += wgt * x.y;
-      acc.z += wgt * x.z;
-      acc.w += wgt * x.w;
-    }
-    __nv_bfloat16* dst = o_lat + ((long long)r * n_h + h) * ATT_DC + d;
-    *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(acc.x, acc.y);
-    *reinterpret_cast<__nv_bfloat162*>(dst + 2) = __floats2bfloat162_rn(acc.z, acc.w);
+  // online log-sum-exp over the parts' lse
+  float mx = -INFINITY, tot = 0.f;
+  for (int s = 0; s < n_parts; ++s) {
+    const float l = lse_part[(long long)(slot0 + s) * n_h + h];
+    const float m2 = fmaxf(mx, l);
+    tot = tot * expf(mx - m2) + expf(l - m2);
+    mx = m2;
   }
-  if (lse && threadIdx.x == 0) lse[(long long)r * n_h + h] = lse_all;
+  const float lse_all = mx + logf(tot);
+  float acc[CPT];
+#pragma unroll
+  for (int e = 0; e < CPT; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int s = 0; s < n_parts; ++s) {
+    const float wgt = expf(lse_part[(long long)(slot0 + s) * n_h + h] - lse_all);
+    const float4* src = reinterpret_cast<const float4*>(o_part + ((long long)(slot0 + s) * n_h + h) * ATT_DC + c0);
+    float4 x[CPT / 4];
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q) x[q] = src[q];
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q) {
+      acc[4 * q] += wgt * x[q].x;
+      acc[4 * q + 1] += wgt * x[q].y;
+      acc[4 * q + 2] += wgt * x[q].z;
+      acc[4 * q + 3] += wgt * x[q].w;
+    }
+  }
+  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((long long)r * n_h + h) * ATT_DC + c0);
+#pragma unroll
+  for (int q = 0; q < CPT / 4; ++q)
+    dst[q] = make_uint2(pack_bf16(acc[4 * q], acc[4 * q + 1]), pack_bf16(acc[4 * q + 2], acc[4 * q + 3]));
+  if (lse && c0 == 0) lse[(long long)r * n_h + h] = lse_all;
 }
 
 }  // namespace mla

@@ -636,9 +636,13 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (p.max_slots > 0) {
-    if (launch_pdl(mla_combine_kernel, dim3(rows * D->n_h), dim3(128), 0, st, 1, (const float*)aw.o_part,
-                   (const float*)aw.lse_part, (const int4*)aw.row_info, D->n_h, (__nv_bfloat16*)o_lat, lse) !=
-        cudaSuccess)
+    // enough blocks for two per SM: split the latent columns when there are few rows
+    const int blocks = rows * (D->n_h / COMBINE_HEADS);
+    const int cs = blocks >= 2 * num_sms() ? 1 : blocks >= num_sms() ? 2 : 4;
+    const dim3 grid(blocks, cs);
+    auto kfn = cs == 1 ? mla_combine_kernel<1> : cs == 2 ? mla_combine_kernel<2> : mla_combine_kernel<4>;
+    if (launch_pdl(kfn, grid, dim3(COMBINE_THREADS), 0, st, 1, (const float*)aw.o_part, (const float*)aw.lse_part,
+                   (const int4*)aw.row_info, D->n_h, (__nv_bfloat16*)o_lat, lse) != cudaSuccess)
       return MLA_ERR_CUDA;
   }
   return MLA_OK;

@@ -22,8 +22,10 @@
  *  - Every tensor argument is a DEVICE pointer owned by the caller; structs
  *    (mla_layer_desc, mla_weights, mla_paged_cache) live in HOST memory and
  *    hold device pointers.  The library never allocates or frees device
- *    memory; scratch comes from the caller's `ws` of at least
- *    mla_workspace_size() bytes (256-byte aligned).
+ *    memory at call time; scratch comes from the caller's `ws` of at least
+ *    mla_workspace_size() bytes (256-byte aligned).  The one exception is
+ *    mla_decode_attn_noalloc, whose scratch is a fixed 32 MiB array that the
+ *    library holds on every device that loads it.
  *  - Row-major layouts.  Weights are [out, in] (the y = W x convention).
  *    Element type is float for MLA_F32 layers and bfloat16 for MLA_BF16
  *    layers, except where a float type is written out (lse, u).
@@ -135,12 +137,14 @@ mla_status_t mla_absorb_q(const mla_layer_desc* desc, const mla_weights* w,
  *   kv_len [B] int32     rows attended by sequence b (including the token just
  *                        appended), 1 <= kv_len[b] <= max_blocks*block_size
  *   num_splits           how the KV rows are cut into work units:
- *                        0 = automatic: all sequences' 128-row tiles are
- *                        spread over about two waves of equal units (a
- *                        sequence is cut only where it is longer than a
- *                        unit); S > 0 = every sequence cut into min(S, its
- *                        tiles) parts.  Cut sequences are merged by a
- *                        log-sum-exp combine.  1 needs no workspace.
+ *                        0 = automatic: the 128-row tiles of all sequences,
+ *                        in sequence order, are dealt to one wave of CTAs
+ *                        (CTA pairs for 128 heads) as equal contiguous
+ *                        ranges, so a sequence is cut wherever a range
+ *                        boundary falls inside it; S > 0 = every sequence
+ *                        cut into min(S, its tiles) parts, one per CTA.
+ *                        Cut sequences are merged by a log-sum-exp combine.
+ *                        1 needs no workspace.
  *   o_lat [B, n_h, d_c]  out: softmax-weighted sum of c^KV (desc dtype)
  *   lse   [B, n_h] float out (may be NULL): natural-log sum of exp(s_j)      */
 mla_status_t mla_decode_attn(const mla_layer_desc* desc, const void* q_lat, const void* q_rope,
@@ -158,8 +162,10 @@ mla_status_t mla_decode_attn(const mla_layer_desc* desc, const void* q_lat, cons
  * Same arguments and results as mla_decode_attn, minus the workspace.  The
  * work-unit list and split partials live in a library-owned device array of
  * 32 MiB (every device that loads the library holds it until the process
- * exits); with num_splits == 0 the automatic plan uses fewer, longer units
- * until they fit, an explicit num_splits whose unit list and partials need
+ * exits); with num_splits == 0 the automatic plan is made for the largest
+ * number of CTAs (CTA pairs) whose unit list and partials fit (63 pairs
+ * instead of 74 for 128 heads at batch 64), an explicit num_splits whose
+ * unit list and partials need
  * more than 32 MiB (about num_splits * B * (n_h * 2052 + 16) bytes, bf16
  * layers) returns MLA_ERR_CAPACITY,
  * as does an fp32 layer whose score scratch (B * n_h * max_blocks *

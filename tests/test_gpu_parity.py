@@ -127,7 +127,7 @@ def test_bf16_other_head_counts(n_h, splits):
     check_decode(w, num_splits=splits)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 5])
+@pytest.mark.parametrize("splits", [1, 2, 4, 5])
 def test_split_count_invariance(splits):
     w = dataclasses.replace(LITE_SMALL, prior="list:300,1500,900,64")
     check_decode(w, num_splits=splits)
@@ -197,25 +197,44 @@ def test_full_size_sampled(name, seqs):
 
 
 def test_long_context_sampled():
+    # 4 x 131072 prior tokens, YaRN s = 40: the appended row (k^R rotated at
+    # position 131072 with the blended frequencies) and the queries of every
+    # sequence, and the whole attention of one sequence.
     w = I.WORKLOADS["long"]
     batch = I.gen_batch(w)
     layer, st = run_gpu(w, batch)
-    ref = O.decode_batch(batch, weights_for(w), seqs=[3], absorbed=True)[0]
+    D, W = w.dims, weights_for(w)
+    rows = new_rows(st, batch)
+    for b in range(w.batch):
+        pos = int(batch.positions[b])
+        assert pos == 131072
+        ref_row = O.compress_kv(D, W, batch.h[b], pos)
+        assert_bf16(rows[b], ref_row, f"cache row {b}")
+        assert_bf16(rows[b][D.d_c:], ref_row[D.d_c:], f"rotated k^R {b}")
+        q_c, q_r = O.queries(D, W, batch.h[b], pos)
+        assert_bf16(np32(st.q_rope)[b], q_r, f"q_rope {b}")
+        assert_bf16(np32(st.q_lat)[b], O.absorb_query(D, W, q_c), f"q_lat {b}")
+    ref = O.decode_batch(batch, W, seqs=[3], absorbed=True)[0]
     assert_bf16(np32(st.o_lat)[3], ref["o_lat"], "o_lat")
+    assert np.max(np.abs(np32(st.lse)[3] - ref["lse"])) < 2e-2
     assert_bf16(np32(st.u)[3], ref["u"], "u")
 
 
-def test_prefill_sampled():
+@pytest.mark.parametrize("b,qs", [(5, [0, 1, 63, 64, 1000, 4095]), (0, [62, 63, 2047, 4094])])
+def test_prefill_sampled(b, qs):
+    # Queries of two of the eight sequences.  With 4096 prior tokens the query
+    # at chunk offset q attends rows 0 .. 4096 + q: q = 63 ends on the last slot
+    # of a page, q = 64 on the first slot of the next, q = 4095 in the last page.
     w = I.WORKLOADS["prefill"]
     batch = I.gen_batch(w)
     layer, st = run_gpu(w, batch)
     D, W = w.dims, weights_for(w)
-    b, n = 5, w.new_tokens
+    n = w.new_tokens
     L = int(batch.prior_len[b])
     prior = O.gather_rows(batch.pool, batch.block_table[b], L, D.block_size)
-    qs = [0, 1, 63, 64, 1000, n - 1]
     new_r, outs = O.prefill_sequence(D, W, batch.h[b * n:(b + 1) * n], L, prior, qs, absorbed=True)
     assert_bf16(new_rows(st, batch)[b * n:(b + 1) * n], new_r, "rows")
     for q in qs:
         assert_bf16(np32(st.o_lat)[b * n + q], outs[q]["o_lat"], f"o_lat q={q}")
+        assert np.max(np.abs(np32(st.lse)[b * n + q] - outs[q]["lse"])) < 2e-2
         assert_bf16(np32(st.u)[b * n + q], outs[q]["u"], f"u q={q}")

@@ -30,7 +30,34 @@ CASES = [
     (dataclasses.replace(LITE, name="lite_auto", batch=4, prior="list:300,1500,900,64"), 0),
     (dataclasses.replace(I.WORKLOADS["v2"], name="v2_splits2", batch=3, prior="list:127,128,3000"), 2),
     (I.WORKLOADS["tiny"], 0),
+    # 128 heads, batch 64, ragged lengths, automatic plan: the plan of a full
+    # wave (74 CTA pairs) needs more than the 32 MiB array, so the entry point
+    # plans for fewer pairs (test_v2_batch64_plan_exceeds_the_array)
+    (dataclasses.replace(I.WORKLOADS["v2"], name="v2_b64_auto"), 0),
 ]
+
+
+def plan_bytes(rows, workers, n_h):
+    """Scratch of an automatic decode plan, carved as the library does: segment
+    list, row table, CTA table, count word, fp32 partials of at
+    most min(rows + workers, 2 * workers) cut segments (each piece 256-byte
+    aligned)."""
+    def take(used, b):
+        return ((used + 255) & ~255) + b
+    units = rows + workers
+    slots = min(units, 2 * workers)
+    u = 0
+    for b in (units * 16, rows * 16, (workers + 1) * 4, 16, slots * n_h * 512 * 4, slots * n_h * 4):
+        u = take(u, b)
+    return u
+
+
+def test_v2_batch64_plan_exceeds_the_array():
+    # one wave of CTA pairs on a 148-SM B200 is 74 pairs; its plan does not fit
+    # 32 MiB, the largest plan that fits has 63 pairs
+    cap = (32 << 20) - 256
+    assert plan_bytes(64, 74, 128) > cap
+    assert max(w for w in range(1, 75) if plan_bytes(64, w, 128) <= cap) == 63
 
 
 @pytest.mark.parametrize("w,splits", CASES, ids=lambda x: getattr(x, "name", str(x)))
@@ -52,7 +79,11 @@ def test_noalloc_matches_workspace_entry_point(w, splits):
         torch.cuda.synchronize()
         assert mla.get_last_error() == 0
         got_o, got_l = o.float().cpu().numpy(), l.cpu().numpy()
-        if w.dims.dtype == "f32":
+        if splits > 0:
+            # explicit split counts: both entry points run the same plan
+            assert np.array_equal(got_o, ref_o), f"o_lat call {call}"
+            assert np.array_equal(got_l, ref_l), f"lse call {call}"
+        elif w.dims.dtype == "f32":
             assert_fp32(got_o, ref_o, f"o_lat call {call}")
             assert_fp32(got_l, ref_l, f"lse call {call}")
         else:
