@@ -2,7 +2,7 @@
 """Benchmark of the MLA decode layer step on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload v2|lite|long|prefill] [--no-cpu-baseline]
+                    [--workload v2|lite|long|prefill] [--no-cpu-baseline] [--no-extra]
 
 A step is one pass of the whole hot path over one batch: compress_append ->
 absorb_q -> decode attention (+ LSE combine) -> out_proj, through the C ABI.
@@ -11,6 +11,12 @@ lengths uniform in [1, 8192] on a randomly permuted page table.  Its cache
 (302 MB) and weights (298 MB) exceed the 126 MB L2, so no flush is needed
 between steps.  Under torchrun each rank runs an independent replica (the
 decode batch shards by sequence; no collective on the data path).
+
+After the headline workload the same run measures the other shapes of the
+scope (V2-Lite decode, 131072-token long-context decode, chunked prefill) and
+adds one block per workload to the same JSON line ("workloads"): tokens/s,
+ms per step, the attention roofline against its binding roof; the headline
+fields are not affected (--no-extra skips them).
 
 --impl reference times the fp64 CPU oracle (the reference arm of this
 comparison) on a bounded sample of the same workload.
@@ -146,6 +152,17 @@ def attention_work(dims, kv_len, rows):
     return bytes_, flops
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_oracle_baseline(w, seconds: float = 12.0):
     """Time the fp64 oracle (un-absorbed form) on whole sequences of the workload
     until `seconds` have passed; tokens/s = decoded tokens / time."""
@@ -178,7 +195,96 @@ def cpu_oracle_baseline(w, seconds: float = 12.0):
             break
     sample = (f"{done} whole sequence(s) of the workload (cache lengths {[int(lens[b]) for b in order[:done]]}), "
               f"fp64 un-absorbed oracle (eqs 9-11 then MHA), numpy BLAS")
-    return {"value": toks / t_total, "unit": "tokens/s", "cores": int(cores), "kind": "oracle", "sample": sample}
+    return {"value": toks / t_total, "unit": "tokens/s", "cores": int(cores), "kind": "oracle", "sample": sample,
+            "cpu_model": cpu_model(), "host_cores": os.cpu_count()}
+
+
+def roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src):
+    """Attention roofline: achieved against the binding roof (the larger of
+    bytes / HBM peak and FLOPs / bf16 peak)."""
+    hbm = float(peaks["hbm_gbs"])
+    tensor = float(peaks["bf16_tflops"])
+    achieved_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
+    achieved_tf = attn_flops / (attn_ms * 1e-3) / 1e12
+    t_hbm, t_tensor = attn_bytes / (hbm * 1e9), attn_flops / (tensor * 1e12)
+    if t_hbm >= t_tensor:
+        roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved_gbs / hbm, 4)}
+    else:
+        roof = {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": tensor, "unit": "TFLOP/s",
+                "frac": round(achieved_tf / tensor, 4)}
+    roof.update({"peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
+                 "other_roof": {"hbm_frac": round(achieved_gbs / hbm, 4), "tensor_frac": round(achieved_tf / tensor, 4),
+                                "attn_bytes_per_launch": attn_bytes, "attn_flops_per_launch": attn_flops,
+                                "attn_us": round(attn_ms * 1e3, 2)}})
+    return roof
+
+
+def workload_work(w, batch):
+    """Algorithmic attention bytes and FLOPs of one step of workload w.  Decode
+    reads every cached row once per sequence; a prefill chunk reads each of its
+    sequences' rows once (all its queries share them) and does the causal
+    query x key products of the latent form."""
+    rows = batch.h.shape[0]
+    if w.new_tokens == 1:
+        return attention_work(w.dims, batch.prior_len + 1, rows)
+    D = w.dims
+    per_q = [int(L) + q + 1 for L in batch.prior_len for q in range(w.new_tokens)]
+    _, flops = attention_work(D, per_q, rows)
+    cached = int(sum(int(L) + w.new_tokens for L in batch.prior_len))
+    bytes_ = cached * D.row * 2 + rows * D.n_h * D.row * 2 + rows * D.n_h * D.d_c * 2
+    return bytes_, flops
+
+
+def measure_extra(name, steps, warmup, dev, peaks, peak_src):
+    """One more workload of the scope in the same run: whole-step and
+    attention-stage device times (CUDA events, max over ranks)."""
+    import torch
+    from head_latent_attention_03_b200 import inputs as I, mla
+    from head_latent_attention_03_b200.layer import MLALayer
+    w = I.WORKLOADS[name]
+    batch = I.gen_batch(w)
+    layer = MLALayer(w.dims, I.gen_weights(w), device=str(dev))
+    st = layer.upload(batch)
+    rows = st.h.shape[0]
+    attn_bytes, attn_flops = workload_work(w, batch)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        layer.step(st)
+    torch.cuda.synchronize()
+    code = mla.get_last_error()
+    if code != 0:
+        raise RuntimeError(f"{name}: device status after warm-up: {mla.status_string(code)}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(steps):
+        layer.compress_append(st)
+        layer.absorb_q(st)
+        ev[k][0].record(stream)
+        layer.attend(st)
+        ev[k][1].record(stream)
+        layer.out_proj(st)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    code = mla.get_last_error()
+    if code != 0:
+        raise RuntimeError(f"{name}: device status after timed steps: {mla.status_string(code)}")
+    t_ms = e0.elapsed_time(e1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    t_ms, attn_ms = max_over_ranks([t_ms, attn_ms], dev)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    out = {"workload": WORKLOAD_TEXT[name], "value": round(world * rows * steps / (t_ms * 1e-3), 1),
+           "unit": "tokens/s", "steps": steps, "warmup": warmup, "ms_per_step": round(t_ms / steps, 4),
+           "roofline": roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src)}
+    out["roofline"]["traffic"] = committed_traffic(name)
+    del layer, st
+    torch.cuda.empty_cache()
+    return out
+
+
+# Steps of the extra workloads (their steps are longer than the headline's).
+EXTRA_STEPS = {"lite": (100, 5), "long": (20, 3), "prefill": (2, 1)}
 
 
 # ---------------------------------------------------------------------------
@@ -221,12 +327,7 @@ def run_ours(args):
     layer = MLALayer(w.dims, W, device=str(dev))
     st = layer.upload(batch)
     rows = st.h.shape[0]
-    kv = (batch.prior_len + 1) if w.new_tokens == 1 else None
-    if w.new_tokens == 1:
-        attn_bytes, attn_flops = attention_work(w.dims, kv, rows)
-    else:
-        per_q = [int(L) + q + 1 for L in batch.prior_len for q in range(w.new_tokens)]
-        attn_bytes, attn_flops = attention_work(w.dims, per_q, rows)
+    attn_bytes, attn_flops = workload_work(w, batch)
     stream = torch.cuda.current_stream()
 
     def step(ev_pair=None):
@@ -309,30 +410,23 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
 
+    peaks, peak_src = load_peaks()
+    extra = {}
+    if not args.no_extra and not args.profile_run:
+        del layer, st
+        torch.cuda.empty_cache()
+        for name in ("lite", "long", "prefill"):
+            if name != args.workload:
+                k, wu = EXTRA_STEPS[name]
+                extra[name] = measure_extra(name, k, wu, dev, peaks, peak_src)
+
     if rank == 0:
-        peaks, peak_src = load_peaks()
-        hbm = float(peaks["hbm_gbs"])
-        tensor = float(peaks["bf16_tflops"])
-        achieved_gbs = attn_bytes / (attn_ms * 1e-3) / 1e9
-        achieved_tf = attn_flops / (attn_ms * 1e-3) / 1e12
-        t_hbm, t_tensor = attn_bytes / (hbm * 1e9), attn_flops / (tensor * 1e12)
-        bound = "hbm" if t_hbm >= t_tensor else "tensor"
+        roof = roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src)
         traffic = committed_traffic(args.workload)
-        if bound == "hbm":
-            roof = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": hbm, "unit": "GB/s",
-                    "frac": round(achieved_gbs / hbm, 4)}
-        else:
-            roof = {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": tensor, "unit": "TFLOP/s",
-                    "frac": round(achieved_tf / tensor, 4)}
         attn_kernel = "mla_attn_pair_kernel" if w.dims.n_h == 128 else "mla_attn_kernel"
         roof.update({"traffic": traffic,
                      "kernel": f"attention stage timed as one: mla_attn_plan_kernel + {attn_kernel} + mla_combine_kernel"
-                               f" (traffic: {attn_kernel} alone)",
-                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback",
-                     "other_roof": {"hbm_frac": round(achieved_gbs / hbm, 4),
-                                    "tensor_frac": round(achieved_tf / tensor, 4),
-                                    "attn_bytes_per_launch": attn_bytes, "attn_flops_per_launch": attn_flops,
-                                    "attn_us": round(attn_ms * 1e3, 2)}})
+                               f" (traffic: {attn_kernel} alone)"})
         value = world * rows * args.steps / (t_ms * 1e-3)
         e2e_value = world * rows * e2e_steps / (t_e2e * 1e-3) if e2e_steps else None
         out = {
@@ -350,6 +444,8 @@ def run_ours(args):
             "gpu_launches": int(n_launch),
             "impl": "ours",
         }
+        if extra:
+            out["workloads"] = extra
         if world == 1 and not args.no_cpu_baseline and not args.profile_run:
             out["cpu_baseline"] = cpu_oracle_baseline(w)
         print(json.dumps(out), flush=True)
@@ -420,6 +516,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["v2", "lite", "long", "prefill"], default="v2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--profile-run", action="store_true",
                     help="only the timed device steps (for ncu launch lists): no clock sampling, e2e or CPU leg")
     args = ap.parse_args()
