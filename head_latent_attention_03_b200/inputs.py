@@ -42,6 +42,12 @@ class LayerDims:
     yarn_beta: float = 32.0
     attn_logit_factor: float = 1.0
     block_size: int = BLOCK
+    # RMSNorm after the compressed latents c^KV and c^Q, then a scale factor
+    # at each of these width bottlenecks (off in the headline workloads)
+    latent_norm: bool = False
+    norm_eps: float = 1e-6
+    scale_kv: float = 1.0
+    scale_q: float = 1.0
 
     @property
     def row(self) -> int:
@@ -86,7 +92,7 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 # tensor ids inside a workload's seed tree
-_T_W = {"w_dkv": 1, "w_kr": 2, "w_dq": 3, "w_uq": 4, "w_qr": 5, "w_uk": 6, "w_uv": 7, "w_o": 8}
+_T_W = {"w_dkv": 1, "w_kr": 2, "w_dq": 3, "w_uq": 4, "w_qr": 5, "w_uk": 6, "w_uv": 7, "w_o": 8, "g_kv": 9, "g_q": 10}
 _T_H, _T_LENS, _T_PRIOR, _T_PERM = 20, 21, 22, 23
 
 
@@ -150,6 +156,12 @@ def gen_weights(w: Workload) -> Dict[str, Optional[np.ndarray]]:
             out[name] = None
             continue
         out[name] = _store(_normal(rng_for(w.cfg_id, _T_W[name]), shp, 1.0 / math.sqrt(shp[1])), D)
+    # RMSNorm gains of the latents: 1 + N(0, 0.1^2) per feature
+    out["g_kv"] = out["g_q"] = None
+    if D.latent_norm:
+        out["g_kv"] = _store(1.0 + _normal(rng_for(w.cfg_id, _T_W["g_kv"]), (D.d_c,), 0.1), D)
+        if D.d_cq:
+            out["g_q"] = _store(1.0 + _normal(rng_for(w.cfg_id, _T_W["g_q"]), (D.d_cq,), 0.1), D)
     return out
 
 

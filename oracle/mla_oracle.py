@@ -31,6 +31,13 @@ explicit choice here, shared by the CUDA path only as a convention):
     window; the logit factor is a parameter (its formula is lost on the page).
   * q^R = RoPE(W^QR c^Q) with c^Q = W^DQ h when queries are compressed, else
     c^Q := h (V2-Lite does not compress queries).
+  * The RMSNorm after the compressed latents and the extra scale factors at
+    these width bottlenecks ([explainer] 3.1.1, no formula printed), when a
+    layer turns them on: c <- s * g * c / sqrt(mean(c^2) + eps) for c^KV
+    (before it is cached) and for c^Q (before W^UQ and W^QR), with per-feature
+    gains g and scalar factors s_kv, s_q.  The factor follows the norm (a
+    factor in front of it would cancel).  k^R is not a compressed latent and
+    is not normalised.
 
 Every function is fp64 and written for clarity, not speed.
 """
@@ -95,17 +102,36 @@ def softmax_scale(D) -> float:
 
 
 # ---------------------------------------------------------------------------
-# projections, [notes] eqs (9), (12), (13); [explainer] 2.2.2
+# projections, [notes] eqs (9), (12), (13); [explainer] 2.2.2, 3.1.1
 # ---------------------------------------------------------------------------
+
+def rms_norm(x: np.ndarray, gain: np.ndarray, eps: float) -> np.ndarray:
+    """gain * x / sqrt(mean(x^2) + eps) over the last axis."""
+    x = np.asarray(x, dtype=F64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return np.asarray(gain, dtype=F64) * x / np.sqrt(ms + eps)
+
+
+def latent_norm(D, W, c: np.ndarray, which: str) -> np.ndarray:
+    """The compressed latent as the layer uses it: RMSNorm plus the bottleneck
+    scale factor when the layer has them ([explainer] 3.1.1), else c."""
+    if not getattr(D, "latent_norm", False):
+        return np.asarray(c, dtype=F64)
+    gain = W["g_kv"] if which == "kv" else W["g_q"]
+    scale = D.scale_kv if which == "kv" else D.scale_q
+    return scale * rms_norm(c, gain, D.norm_eps)
+
 
 def compress_kv(D, W: Dict[str, np.ndarray], h_t: np.ndarray, pos: int) -> np.ndarray:
     """The cached row of token t: [c^KV_t ; k^R_t].
 
-    c^KV_t = W^DKV h_t (eq 9).  k^R_t = RoPE_pos(W^KR h_t): the shared RoPE
-    key comes straight from h_t, not from the latent ([explainer] 2.2.2).
+    c^KV_t = W^DKV h_t (eq 9), normalised and scaled when the layer has the
+    latent RMSNorm ([explainer] 3.1.1).  k^R_t = RoPE_pos(W^KR h_t): the
+    shared RoPE key comes straight from h_t, not from the latent
+    ([explainer] 2.2.2).
     """
     h = np.asarray(h_t, dtype=F64)
-    c_kv = W["w_dkv"].astype(F64) @ h
+    c_kv = latent_norm(D, W, W["w_dkv"].astype(F64) @ h, "kv")
     k_r = rope_rotate(W["w_kr"].astype(F64) @ h, pos, dims_theta(D))
     return np.concatenate([c_kv, k_r])
 
@@ -117,7 +143,7 @@ def queries(D, W: Dict[str, np.ndarray], h_t: np.ndarray, pos: int) -> Tuple[np.
     q^C = W^UQ c^Q (eq 13); q^R_i = RoPE_pos(W^QR_i c^Q) ([explainer] 2.2.2).
     """
     h = np.asarray(h_t, dtype=F64)
-    c_q = W["w_dq"].astype(F64) @ h if D.d_cq else h
+    c_q = latent_norm(D, W, W["w_dq"].astype(F64) @ h, "q") if D.d_cq else h
     q_c = (W["w_uq"].astype(F64) @ c_q).reshape(D.n_h, D.d_h)
     q_r_pre = (W["w_qr"].astype(F64) @ c_q).reshape(D.n_h, D.d_hr)
     q_r = rope_rotate(q_r_pre, pos, dims_theta(D))

@@ -361,3 +361,77 @@ def test_vanishing_queries_attend_uniformly_over_all_visible_rows():
         for i in range(D.n_h):
             np.testing.assert_allclose(out["o_lat"][i], want, rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(out["lse"], math.log(L + 1), rtol=1e-12)
+
+
+# RMSNorm after the compressed latents and the bottleneck scale factors
+# ([explainer] 3.1.1, no formula printed; the reading: c <- s * g * c / rms(c)).
+NORM_DIMS = LayerDims(d=40, n_h=2, d_h=8, d_c=24, d_cq=20, d_hr=6, dtype="f32", latent_norm=True, norm_eps=0.0,
+                      scale_kv=1.7, scale_q=0.6)
+
+
+def _norm_weights(D, rng, gains=True):
+    W = _rand_weights(D, rng)
+    W["g_kv"] = 1.0 + 0.1 * rng.standard_normal(D.d_c) if gains else np.ones(D.d_c)
+    W["g_q"] = 1.0 + 0.1 * rng.standard_normal(D.d_cq) if gains else np.ones(D.d_cq)
+    return W
+
+
+def test_latent_norm_gives_the_scale_as_rms():
+    # unit gains, eps = 0: the cached latent's root mean square is exactly the
+    # bottleneck scale factor, whatever h is; the factor acts after the norm,
+    # so doubling it doubles the latent
+    rng = np.random.default_rng(31)
+    D = NORM_DIMS
+    W = _norm_weights(D, rng, gains=False)
+    for _ in range(3):
+        h = rng.standard_normal(D.d) * rng.uniform(0.1, 10.0)
+        c = O.compress_kv(D, W, h, 5)[:D.d_c]
+        assert abs(math.sqrt(np.mean(c * c)) - D.scale_kv) < 1e-12
+        D2 = LayerDims(**{**D.__dict__, "scale_kv": 2 * D.scale_kv})
+        assert np.allclose(O.compress_kv(D2, W, h, 5)[:D.d_c], 2 * c, rtol=1e-13, atol=0)
+
+
+def test_latent_norm_removes_the_scale_of_h_but_not_from_k_rope():
+    # c^KV and c^Q are linear in h; after the norm (eps = 0) they no longer
+    # depend on h's scale, so neither do q^C and q^R.  k^R comes from h
+    # directly and scales with it.
+    rng = np.random.default_rng(32)
+    D = NORM_DIMS
+    W = _norm_weights(D, rng)
+    h = rng.standard_normal(D.d)
+    a = 3.25
+    r1, r2 = O.compress_kv(D, W, h, 9), O.compress_kv(D, W, a * h, 9)
+    assert np.allclose(r2[:D.d_c], r1[:D.d_c], rtol=1e-12, atol=0)
+    assert np.allclose(r2[D.d_c:], a * r1[D.d_c:], rtol=1e-12, atol=0)
+    (qc1, qr1), (qc2, qr2) = O.queries(D, W, h, 9), O.queries(D, W, a * h, 9)
+    assert np.allclose(qc2, qc1, rtol=1e-12, atol=1e-14) and np.allclose(qr2, qr1, rtol=1e-12, atol=1e-14)
+    # without the norm the queries scale with h
+    D0 = LayerDims(**{**D.__dict__, "latent_norm": False})
+    qc0a, _ = O.queries(D0, W, h, 9)
+    qc0b, _ = O.queries(D0, W, a * h, 9)
+    assert np.allclose(qc0b, a * qc0a, rtol=1e-12, atol=1e-14)
+
+
+def test_latent_norm_gain_is_per_feature():
+    # eps = 0: the latent with gains g, divided feature by feature by the
+    # latent with unit gains, is g itself
+    rng = np.random.default_rng(33)
+    D = NORM_DIMS
+    W = _norm_weights(D, rng)
+    W1 = dict(W, g_kv=np.ones(D.d_c), g_q=np.ones(D.d_cq))
+    h = rng.standard_normal(D.d)
+    assert np.allclose(O.compress_kv(D, W, h, 2)[:D.d_c] / O.compress_kv(D, W1, h, 2)[:D.d_c], W["g_kv"],
+                       rtol=1e-12, atol=0)
+
+
+def test_latent_norm_epsilon_closed_form():
+    # unit gains and factors: mean(y^2) = m / (m + eps), m = mean(c^2) of the
+    # raw latent W^DKV h
+    rng = np.random.default_rng(34)
+    D = LayerDims(**{**NORM_DIMS.__dict__, "norm_eps": 0.05, "scale_kv": 1.0})
+    W = _norm_weights(D, rng, gains=False)
+    h = 0.2 * rng.standard_normal(D.d)
+    raw = W["w_dkv"] @ h
+    m = float(np.mean(raw * raw))
+    y = O.compress_kv(D, W, h, 0)[:D.d_c]
+    assert abs(float(np.mean(y * y)) - m / (m + D.norm_eps)) < 1e-13

@@ -41,6 +41,18 @@ MUTATIONS = {
     # paged-cache gather reading the neighbouring slot of each page
     "gather_slot_shift": ("out[j] = pool[table_row[j // block], j % block]",
                           "out[j] = pool[table_row[j // block], (j + 1) % block]"),
+    # latent RMSNorm dividing by the sum of squares instead of their mean
+    "norm_sum_not_mean": ("ms = np.mean(x * x, axis=-1, keepdims=True)", "ms = np.sum(x * x, axis=-1, keepdims=True)"),
+    # latent RMSNorm without its gains
+    "norm_gain_dropped": ("return np.asarray(gain, dtype=F64) * x / np.sqrt(ms + eps)",
+                          "return x / np.sqrt(ms + eps)"),
+    # epsilon added outside the square root
+    "norm_eps_outside": ("x / np.sqrt(ms + eps)", "x / (np.sqrt(ms) + eps)"),
+    # bottleneck scale factor dropped
+    "norm_scale_dropped": ("return scale * rms_norm(c, gain, D.norm_eps)", "return rms_norm(c, gain, D.norm_eps)"),
+    # query latent left un-normalised
+    "norm_query_skipped": ("c_q = latent_norm(D, W, W[\"w_dq\"].astype(F64) @ h, \"q\") if D.d_cq else h",
+                           "c_q = W[\"w_dq\"].astype(F64) @ h if D.d_cq else h"),
     # W^O applied before W^UV's head split is undone
     "out_proj_heads": ("o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64))",
                        "o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64)[::-1])"),
