@@ -34,6 +34,7 @@ bool desc_valid(const mla_layer_desc* D) {
   if (D->d_hr % 2 != 0 || D->block_size <= 0) return false;
   if (!(D->rope_base > 0.0) || !(D->yarn_scale >= 1.0) || !(D->attn_logit_factor > 0.0)) return false;
   if (D->yarn_scale > 1.0 && (D->yarn_orig_ctx <= 0 || !(D->yarn_beta > D->yarn_alpha))) return false;
+  if (D->latent_norm && (!(D->norm_eps >= 0.0) || !(D->scale_kv > 0.0) || !(D->scale_q > 0.0))) return false;
   return D->dtype == MLA_F32 || D->dtype == MLA_BF16;
 }
 
@@ -66,6 +67,10 @@ F32Layer f32_layer(const mla_layer_desc* D) {
   L.block_size = D->block_size;
   L.rope = rope_params(D);
   L.scale_log2 = (float)(softmax_scale(D) * 1.4426950408889634);
+  L.latent_norm = D->latent_norm ? 1 : 0;
+  L.norm_eps = (float)D->norm_eps;
+  L.scale_kv = (float)D->scale_kv;
+  L.scale_q = (float)D->scale_q;
   return L;
 }
 
@@ -138,7 +143,8 @@ size_t mla_workspace_size(const mla_layer_desc* D, int T, int B, int max_kv_len)
 mla_status_t mla_compress_append(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* seq_idx,
                                  const int32_t* pos, int T, mla_paged_cache* cache, void* ws, size_t ws_bytes,
                                  void* stream) {
-  if (!desc_valid(D) || !w || !w->w_dkv || !w->w_kr || !h || !seq_idx || !pos || T < 0 || !cache_valid(cache))
+  if (!desc_valid(D) || !w || !w->w_dkv || !w->w_kr || !h || !seq_idx || !pos || T < 0 || !cache_valid(cache) ||
+      (D->latent_norm && !w->g_kv))
     return MLA_ERR_INVALID_ARG;
   if (T == 0) return MLA_OK;
   if (D->dtype == MLA_F32) {
@@ -147,7 +153,8 @@ mla_status_t mla_compress_append(const mla_layer_desc* D, const mla_weights* w, 
     if (smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
     MLA_COUNT_LAUNCH();
     f32_compress_append_kernel<<<T, 256, smem, as_stream(stream)>>>(
-        L, (const float*)h, (const float*)w->w_dkv, (const float*)w->w_kr, seq_idx, pos, (float*)cache->pool,
+        L, (const float*)h, (const float*)w->w_dkv, (const float*)w->w_kr, (const float*)w->g_kv, seq_idx, pos,
+        (float*)cache->pool,
         cache->num_blocks, cache->block_table, cache->max_blocks);
     return check_launch();
   }
@@ -158,7 +165,7 @@ mla_status_t mla_compress_append(const mla_layer_desc* D, const mla_weights* w, 
 mla_status_t mla_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos, int T,
                           void* q_lat, void* q_rope, void* ws, size_t ws_bytes, void* stream) {
   if (!desc_valid(D) || !w || !w->w_uq || !w->w_qr || !w->w_uk || (D->d_cq && !w->w_dq) || !h || !pos || T < 0 ||
-      !q_lat || !q_rope)
+      !q_lat || !q_rope || (D->latent_norm && D->d_cq && !w->g_q))
     return MLA_ERR_INVALID_ARG;
   if (T == 0) return MLA_OK;
   if (D->dtype == MLA_F32) {
@@ -170,7 +177,8 @@ mla_status_t mla_absorb_q(const mla_layer_desc* D, const mla_weights* w, const v
       cudaFuncSetAttribute(f32_absorb_q_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     MLA_COUNT_LAUNCH();
     f32_absorb_q_kernel<<<T, 256, smem, as_stream(stream)>>>(L, (const float*)h, (const float*)w->w_dq,
-                                                               (const float*)w->w_uq, (const float*)w->w_qr,
+                                                               (const float*)w->g_q, (const float*)w->w_uq,
+                                                               (const float*)w->w_qr,
                                                                (const float*)w->w_uk, pos, (float*)q_lat,
                                                                (float*)q_rope);
     return check_launch();

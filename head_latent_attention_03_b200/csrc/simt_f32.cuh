@@ -14,7 +14,30 @@ struct F32Layer {
   int d, n_h, d_h, d_c, d_cq, d_hr, block_size;
   RopeParams rope;
   float scale_log2;  // softmax scale * log2(e)
+  int latent_norm;   // RMSNorm + scale factor on c^KV and c^Q
+  float norm_eps, scale_kv, scale_q;
 };
+
+// v[0..n) <- scale * g * v / sqrt(mean(v^2) + eps) over the block (the
+// latent RMSNorm with its bottleneck scale factor, DeepSeek-V2 explainer,
+// adg.csdn.net, section 3.1.1).  All threads of the block call it.
+__device__ void f32_rmsnorm_inplace(float* v, int n, const float* __restrict__ g, float eps, float scale) {
+  __shared__ float part[32];
+  __shared__ float inv;
+  float acc = 0.f;
+  for (int k = threadIdx.x; k < n; k += blockDim.x) acc = fmaf(v[k], v[k], acc);
+  acc = warp_sum(acc);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += part[w];
+    inv = 1.f / sqrtf(tot / (float)n + eps);
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < n; k += blockDim.x) v[k] = scale * g[k] * (v[k] * inv);
+  __syncthreads();
+}
 
 // y[r] = sum_k W[r, k] x[k] for r in [0, rows), one warp per row.
 __device__ __forceinline__ void f32_matvec_warp(const float* __restrict__ W, const float* x, float* y, int rows,
@@ -42,7 +65,8 @@ __device__ __forceinline__ void f32_rope_inplace(float* v, int d_hr, long long p
 
 // One block per new token: [c^KV ; RoPE(W^KR h)] -> its cache slot.
 __global__ void f32_compress_append_kernel(F32Layer L, const float* __restrict__ h, const float* __restrict__ w_dkv,
-                                           const float* __restrict__ w_kr, const int32_t* __restrict__ seq_idx,
+                                           const float* __restrict__ w_kr, const float* __restrict__ g_kv,
+                                           const int32_t* __restrict__ seq_idx,
                                            const int32_t* __restrict__ pos, float* __restrict__ pool, int num_blocks,
                                            const int32_t* __restrict__ table, int max_blocks) {
   extern __shared__ float sm[];
@@ -55,6 +79,7 @@ __global__ void f32_compress_append_kernel(F32Layer L, const float* __restrict__
   f32_matvec_warp(w_dkv, x, y, L.d_c, L.d);
   f32_matvec_warp(w_kr, x, y + L.d_c, L.d_hr, L.d);
   __syncthreads();
+  if (L.latent_norm) f32_rmsnorm_inplace(y, L.d_c, g_kv, L.norm_eps, L.scale_kv);
   const long long p = pos[t];
   f32_rope_inplace(y + L.d_c, L.d_hr, p, L.rope);
   __syncthreads();
@@ -71,7 +96,8 @@ __global__ void f32_compress_append_kernel(F32Layer L, const float* __restrict__
 
 // One block per token: q_lat = (W^UK_i)^T W^UQ_i c^Q and q_rope = RoPE(W^QR_i c^Q).
 __global__ void f32_absorb_q_kernel(F32Layer L, const float* __restrict__ h, const float* __restrict__ w_dq,
-                                    const float* __restrict__ w_uq, const float* __restrict__ w_qr,
+                                    const float* __restrict__ g_q, const float* __restrict__ w_uq,
+                                    const float* __restrict__ w_qr,
                                     const float* __restrict__ w_uk, const int32_t* __restrict__ pos,
                                     float* __restrict__ q_lat, float* __restrict__ q_rope) {
   extern __shared__ float sm[];
@@ -89,6 +115,7 @@ __global__ void f32_absorb_q_kernel(F32Layer L, const float* __restrict__ h, con
     for (int k = threadIdx.x; k < L.d; k += blockDim.x) cq[k] = x[k];
   }
   __syncthreads();
+  if (L.d_cq && L.latent_norm) f32_rmsnorm_inplace(cq, L.d_cq, g_q, L.norm_eps, L.scale_q);
   f32_matvec_warp(w_uq, cq, qc, L.n_h * L.d_h, q_in);
   f32_matvec_warp(w_qr, cq, qr, L.n_h * L.d_hr, q_in);
   __syncthreads();

@@ -50,6 +50,7 @@ struct GemmEpi {
   int d_hr;
   // EPI_CACHE
   int d_c;
+  float* lat_f32;            // non-null: c^KV goes here ([t][d_c] fp32) for the latent RMSNorm, not to the cache
   const int32_t* seq_idx;    // [T]
   __nv_bfloat16* pool;
   int num_blocks, max_blocks, block_size;
@@ -115,6 +116,10 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
     case EPI_CACHE: {
       const int row = e.d_c + e.d_hr;
       const long long p = e.pos[t];
+      if (n < e.d_c && e.lat_f32) {
+        *reinterpret_cast<float2*>(e.lat_f32 + (long long)t * e.d_c + n) = v;
+        break;
+      }
       if (n >= e.d_c) {
         float c, s;
         rope_cos_sin_reduced(e.rope.theta[(n - e.d_c) / 2], p, &c, &s);

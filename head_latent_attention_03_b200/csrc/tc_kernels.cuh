@@ -16,6 +16,7 @@
 
 #include "../../include/mla.h"
 #include "common.cuh"
+#include "norm.cuh"
 #include "rope.cuh"
 #include "tc_attn.cuh"
 #include "tc_attn2.cuh"
@@ -294,10 +295,13 @@ inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
 
 // Workspace of the projections: only the bf16 intermediates between two
 // GEMMs (K splits are reduced inside each GEMM's cluster).
-inline size_t ws_compress(const mla_layer_desc*, int) { return 0; }
+inline size_t ws_compress(const mla_layer_desc* D, int T) {
+  return D->latent_norm ? (size_t)T * D->d_c * 4 + 256 : 0;
+}
 inline size_t ws_absorb(const mla_layer_desc* D, int T) {
   Carver c{nullptr, 0};
   if (D->d_cq) c.take((size_t)T * D->d_cq * 2);
+  if (D->d_cq && D->latent_norm) c.take((size_t)T * D->d_cq * 4);
   c.take((size_t)T * D->n_h * D->d_h * 2);
   return c.used;
 }
@@ -408,9 +412,16 @@ static Carver carve(void* ws, size_t ws_bytes) {
 
 static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weights* w, const void* h,
                                        const int32_t* seq_idx, const int32_t* pos, int T, mla_paged_cache* cache,
-                                       void*, size_t, cudaStream_t st) {
-  if (!aligned16(h) || !aligned16(w->w_dkv) || !aligned16(w->w_kr) || !aligned16(cache->pool))
+                                       void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!aligned16(h) || !aligned16(w->w_dkv) || !aligned16(w->w_kr) || !aligned16(cache->pool) ||
+      (D->latent_norm && !aligned16(w->g_kv)))
     return MLA_ERR_INVALID_ARG;
+  float* lat = nullptr;  // fp32 c^KV for the latent RMSNorm
+  if (D->latent_norm) {
+    Carver cv = carve(ws, ws_bytes);
+    lat = (float*)cv.take((size_t)T * D->d_c * 4);
+    if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  }
   // [c^KV ; k^R] = [W^DKV ; W^KR] h  (eq 9 + decoupled key), RoPE on k^R,
   // bf16 rows scattered into the paged cache
   GemmCall c{};
@@ -437,19 +448,40 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   e.max_blocks = cache->max_blocks;
   e.block_size = D->block_size;
   e.table = cache->block_table;
-  return run_gemm(c, e, plan_compress(D, T), st);
+  e.lat_f32 = lat;
+  mla_status_t s = run_gemm(c, e, plan_compress(D, T), st);
+  if (s != MLA_OK || !lat) return s;
+  // c^KV <- scale_kv * g_kv * c^KV / rms(c^KV), into the cache row
+  NormArgs na{};
+  na.x = lat;
+  na.n = D->d_c;
+  na.gain = (const __nv_bfloat16*)w->g_kv;
+  na.eps = (float)D->norm_eps;
+  na.scale = (float)D->scale_kv;
+  na.pool = (__nv_bfloat16*)cache->pool;
+  na.table = cache->block_table;
+  na.seq_idx = seq_idx;
+  na.pos = pos;
+  na.num_blocks = cache->num_blocks;
+  na.max_blocks = cache->max_blocks;
+  na.block_size = D->block_size;
+  na.row = D->d_c + D->d_hr;
+  return launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) == cudaSuccess ? MLA_OK
+                                                                                                      : MLA_ERR_CUDA;
 }
 
 static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos,
                                 int T, void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (!aligned16(h) || !aligned16(w->w_uq) || !aligned16(w->w_qr) || !aligned16(w->w_uk) ||
-      (D->d_cq && !aligned16(w->w_dq)) || !aligned16(q_lat) || !aligned16(q_rope))
+      (D->d_cq && !aligned16(w->w_dq)) || !aligned16(q_lat) || !aligned16(q_rope) ||
+      (D->d_cq && D->latent_norm && !aligned16(w->g_q)))
     return MLA_ERR_INVALID_ARG;
   Carver cv = carve(ws, ws_bytes);
   const int nq = D->n_h * D->d_h, nr = D->n_h * D->d_hr;
   const int q_in = D->d_cq ? D->d_cq : D->d;
   __nv_bfloat16* cq = D->d_cq ? (__nv_bfloat16*)cv.take((size_t)T * D->d_cq * 2) : nullptr;
   __nv_bfloat16* qc = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
+  float* cq32 = D->d_cq && D->latent_norm ? (float*)cv.take((size_t)T * D->d_cq * 4) : nullptr;
   if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   mla_status_t s;
   const void* qsrc = h;
@@ -465,10 +497,27 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     c.T = T;
     c.Z = 1;
     GemmEpi e{};
-    e.kind = EPI_BF16;
-    e.out = cq;
+    if (cq32) {  // fp32 c^Q, then the latent RMSNorm writes the bf16 c^Q
+      e.kind = EPI_F32;
+      e.out = cq32;
+    } else {
+      e.kind = EPI_BF16;
+      e.out = cq;
+    }
     e.out_t = D->d_cq;
     if ((s = run_gemm(c, e, plan_q1(D, T), st)) != MLA_OK) return s;
+    if (cq32) {
+      NormArgs na{};
+      na.x = cq32;
+      na.n = D->d_cq;
+      na.gain = (const __nv_bfloat16*)w->g_q;
+      na.eps = (float)D->norm_eps;
+      na.scale = (float)D->scale_q;
+      na.out = cq;
+      na.out_t = D->d_cq;
+      if (launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    }
     qsrc = cq;
   }
   {  // [q^C ; q^R] = [W^UQ ; W^QR] c^Q   (eq 13 + decoupled query), RoPE on q^R

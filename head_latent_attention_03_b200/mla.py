@@ -30,11 +30,13 @@ class LayerDesc(ctypes.Structure):
                 ("d_cq", ctypes.c_int), ("d_hr", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("rope_base", ctypes.c_double), ("yarn_scale", ctypes.c_double),
                 ("yarn_orig_ctx", ctypes.c_int), ("yarn_alpha", ctypes.c_double), ("yarn_beta", ctypes.c_double),
-                ("attn_logit_factor", ctypes.c_double)]
+                ("attn_logit_factor", ctypes.c_double), ("latent_norm", ctypes.c_int), ("norm_eps", ctypes.c_double),
+                ("scale_kv", ctypes.c_double), ("scale_q", ctypes.c_double)]
 
 
 class Weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("w_dkv", "w_kr", "w_dq", "w_uq", "w_qr", "w_uk", "w_uv", "w_o")]
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_dkv", "w_kr", "w_dq", "w_uq", "w_qr", "w_uk", "w_uv", "w_o",
+                                                "g_kv", "g_q")]
 
 
 class PagedCache(ctypes.Structure):
@@ -97,7 +99,9 @@ def layer_desc(dims) -> LayerDesc:
     """LayerDesc from any object with the mla_layer_desc field names (e.g. inputs.LayerDims)."""
     return LayerDesc(dims.d, dims.n_h, dims.d_h, dims.d_c, dims.d_cq, dims.d_hr, dims.block_size,
                      MLA_BF16 if dims.dtype == "bf16" else MLA_F32, dims.rope_base, dims.yarn_scale,
-                     dims.yarn_orig_ctx, dims.yarn_alpha, dims.yarn_beta, dims.attn_logit_factor)
+                     dims.yarn_orig_ctx, dims.yarn_alpha, dims.yarn_beta, dims.attn_logit_factor,
+                     int(getattr(dims, "latent_norm", False)), getattr(dims, "norm_eps", 0.0),
+                     getattr(dims, "scale_kv", 1.0), getattr(dims, "scale_q", 1.0))
 
 
 def _ptr(t) -> Optional[int]:
@@ -112,7 +116,8 @@ def _stream(stream) -> Optional[int]:
 
 
 def weights(w: dict) -> Weights:
-    return Weights(*[_ptr(w.get(n)) for n in ("w_dkv", "w_kr", "w_dq", "w_uq", "w_qr", "w_uk", "w_uv", "w_o")])
+    return Weights(*[_ptr(w.get(n)) for n in ("w_dkv", "w_kr", "w_dq", "w_uq", "w_qr", "w_uk", "w_uv", "w_o",
+                                               "g_kv", "g_q")])
 
 
 def paged_cache(pool, block_table) -> PagedCache:

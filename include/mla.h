@@ -85,15 +85,26 @@ typedef struct {
   int yarn_orig_ctx;         /* original context window of the YaRN blend */
   double yarn_alpha, yarn_beta;
   double attn_logit_factor;  /* multiplies every logit; 1 when YaRN is off */
+  /* RMSNorm after the compressed latents and a scale factor at each of these
+   * width bottlenecks (DeepSeek-V2 explainer, section 3.1.1):
+   *   c^KV <- scale_kv * g_kv * c^KV / sqrt(mean(c^KV^2) + norm_eps), before it is cached
+   *   c^Q  <- scale_q  * g_q  * c^Q  / sqrt(mean(c^Q^2)  + norm_eps), before W^UQ, W^QR
+   * (c^Q only when d_cq > 0).  0 = off: the other three fields are ignored. */
+  int latent_norm;
+  double norm_eps;           /* >= 0 */
+  double scale_kv, scale_q;  /* > 0 */
 } mla_layer_desc;
 
 /* Projection matrices, [out, in] row-major, element type = desc.dtype.
  *   w_dkv [d_c, d]            w_kr [d_hr, d]          w_dq [d_cq, d] (NULL if d_cq == 0)
  *   w_uq  [n_h*d_h, q_in]     w_qr [n_h*d_hr, q_in]   (q_in = d_cq, or d when d_cq == 0)
  *   w_uk  [n_h*d_h, d_c]      w_uv [n_h*d_h, d_c]     (head i = rows i*d_h .. i*d_h+d_h-1)
- *   w_o   [d, n_h*d_h]                                                            */
+ *   w_o   [d, n_h*d_h]
+ *   g_kv  [d_c], g_q [d_cq]   RMSNorm gains of the latents (read only when
+ *                             desc.latent_norm; g_q only when d_cq > 0)        */
 typedef struct {
   const void *w_dkv, *w_kr, *w_dq, *w_uq, *w_qr, *w_uk, *w_uv, *w_o;
+  const void *g_kv, *g_q;
 } mla_weights;
 
 /* Paged latent cache: pool [num_blocks, block_size, d_c + d_hr]; token j of

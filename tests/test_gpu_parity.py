@@ -118,6 +118,21 @@ def test_bf16_small(w):
     check_decode(w)
 
 
+def _with_norm(w, name):
+    # RMSNorm after c^KV and c^Q with gains 1 + N(0, 0.1^2) and bottleneck
+    # scale factors away from 1
+    return dataclasses.replace(w, name=name, dims=dataclasses.replace(w.dims, latent_norm=True, norm_eps=1e-6,
+                                                                      scale_kv=1.5, scale_q=0.75))
+
+
+@pytest.mark.parametrize("w", [_with_norm(I.WORKLOADS["tiny"], "tiny_norm"), _with_norm(LITE_SMALL, "lite_norm"),
+                               _with_norm(V2_SMALL, "v2_norm")], ids=lambda w: w.name)
+def test_latent_norm(w):
+    # the cached c^KV row, q_lat (from the normalised c^Q) and the whole
+    # layer against the oracle with the same norm
+    check_decode(w)
+
+
 @pytest.mark.parametrize("n_h,splits", [(32, 0), (32, 3), (64, 0), (64, 3)])
 def test_bf16_other_head_counts(n_h, splits):
     # 32 and 64 heads: the one-CTA kernel with one or two 32-head groups per
