@@ -250,6 +250,26 @@ mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* D, const void* q_lat,
                       o_lat, lse, as_stream(stream), workers);
 }
 
+mla_status_t mla_decode_attn_partial(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
+                                     const mla_paged_cache* cache, const int32_t* kv_begin, const int32_t* kv_end,
+                                     int B, void* ws, size_t ws_bytes, float* o_part, float* lse_part, void* stream) {
+  if (!desc_valid(D) || !q_lat || !q_rope || !cache_valid(cache) || !kv_begin || !kv_end || B < 0 || !o_part ||
+      !lse_part)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (D->dtype != MLA_BF16 || !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_attention(D, q_lat, q_rope, cache, kv_end, nullptr, 1, B, ws, ws_bytes, 0, nullptr, lse_part,
+                      as_stream(stream), 0, kv_begin, o_part);
+}
+
+mla_status_t mla_lse_merge(const mla_layer_desc* D, const float* o_parts, const float* lse_parts, int R, int B,
+                           void* o_lat, float* lse, void* stream) {
+  if (!desc_valid(D) || !o_parts || !lse_parts || R < 1 || B < 0 || !o_lat) return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if (D->dtype == MLA_BF16 && !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_lse_merge(D, o_parts, lse_parts, R, B, o_lat, lse, as_stream(stream));
+}
+
 mla_status_t mla_prefill_attn(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
                               const mla_paged_cache* cache, const int32_t* q_start, int q_per_seq, int B, void* ws,
                               size_t ws_bytes, void* o_lat, float* lse, void* stream) {

@@ -77,7 +77,8 @@ struct AttnArgs {
   float scale_log2;
   const int32_t* table;
   const uint8_t* pool;     // cache pages, 64 rows x 1152 bytes each (L2 prefetch)
-  const int32_t* kv_len;   // decode: per row; nullptr for prefill
+  const int32_t* kv_len;   // decode: per row (the end of the row's range); nullptr for prefill
+  const int32_t* kv_begin; // partial decode: first row of each row's range (multiple of 128); else nullptr
   const int32_t* q_start;  // prefill: per sequence
   const int4* units;       // [segment] {row, first token, end token, partial slot or -1 (whole row)};
                            // nullptr: CTA w does all of row w
@@ -118,7 +119,8 @@ __device__ __forceinline__ SegInfo att_seg_info(const AttnArgs& a, int s) {
   S.t_end = u.z;
   S.pslot = u.w;
   S.kv = att_kv_len(a, S.r);
-  const bool ok = S.kv >= 1 && S.kv <= a.max_blocks * 64;
+  // a partial decode may give a row an empty range (kv_end == kv_begin, 0 included)
+  const bool ok = S.kv >= (a.kv_begin ? 0 : 1) && S.kv <= a.max_blocks * 64;
   if (!ok) record_error(ERR_CAPACITY, 401);
   S.n_tiles = ok && S.t_end > S.t_begin ? (S.t_end - S.t_begin + ATT_TILE - 1) / ATT_TILE : 0;
   return S;
@@ -169,6 +171,9 @@ struct TileCursor {
 //     that straddles range boundaries becomes several segments.
 //   explicit (splits > 0): every row cut into min(splits, its tiles) equal
 //     segments, one per CTA.
+// With kv_begin (partial decode) row b covers rows [kv_begin[b], kv_len[b])
+// only, in tiles from kv_begin[b] (a multiple of 128), and force_slots gives
+// every segment a partial slot: the combine then writes every row in fp32.
 // Segments of rows cut in several get partial slots (merged by the combine
 // kernel); the others write their output directly.  Outputs:
 //   units[u]    = {row, first token, end token, slot or -1}   (row order)
@@ -177,7 +182,8 @@ struct TileCursor {
 __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const int32_t* __restrict__ q_start,
                                      int q_per_seq, int rows, int max_len, int workers, int splits, int max_units,
                                      int max_slots, int4* __restrict__ units, int4* __restrict__ row_info,
-                                     int* __restrict__ work, int* __restrict__ n_units) {
+                                     int* __restrict__ work, int* __restrict__ n_units,
+                                     const int32_t* __restrict__ kv_begin, int force_slots) {
   __shared__ long long s_sum[32];
   __shared__ int s_scan[3][1024];
   __shared__ int s_lastw[1024];
@@ -189,7 +195,21 @@ __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const i
     const int kv = kv_len ? kv_len[b] : q_start[b / q_per_seq] + b % q_per_seq + 1;
     return min(max(kv, 0), max_len);
   };
-  auto tiles_of = [&](int b) -> int { return (kv_of(b) + ATT_TILE - 1) / ATT_TILE; };
+  // first row of b's range; a kv_begin that is not a multiple of 128 or lies
+  // outside [0, kv] empties the row and is reported
+  auto kb_of = [&](int b) -> int {
+    if (!kv_begin) return 0;
+    const int kb = kv_begin[b], kv = kv_of(b);
+    if (kb < 0 || kb % ATT_TILE != 0 || kb > kv) {
+      record_error(ERR_CAPACITY, 404);
+      return kv;
+    }
+    return kb;
+  };
+  auto tiles_of = [&](int b) -> int {
+    const int kb = kb_of(b);
+    return (kv_of(b) - kb + ATT_TILE - 1) / ATT_TILE;
+  };
   long long local = 0;
   for (int b = tid; b < rows; b += nt) local += tiles_of(b);
   for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
@@ -237,7 +257,7 @@ __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const i
     const int t_last = s_scan[0][nt - 1];
     __syncthreads();
     s_scan[1][tid] = parts;
-    s_scan[2][tid] = parts > 1 ? parts : 0;
+    s_scan[2][tid] = (parts > 1 || force_slots) ? parts : 0;
     __syncthreads();
     for (int off = 1; off < nt; off <<= 1) {
       const int a1 = tid >= off ? s_scan[1][tid - off] : 0;
@@ -248,18 +268,19 @@ __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const i
       __syncthreads();
     }
     const int u0 = run_units + s_scan[1][tid] - parts;
-    const int sl0 = parts > 1 ? run_slots + s_scan[2][tid] - parts : -1;
+    const bool slotted = parts > 1 || force_slots;
+    const int sl0 = slotted ? run_slots + s_scan[2][tid] - parts : -1;
     const bool over = b < rows && (u0 + parts > max_units || sl0 + parts > max_slots ||
                                    (splits == 0 && lastw >= workers));
     if (over) record_error(ERR_CAPACITY, 402);  // beyond the host's bounds: cannot happen for a valid plan
     bad |= over;
     if (b < rows && !over) {
       row_info[b] = make_int4(u0, parts, sl0, 0);
-      const int kv = kv_of(b);
+      const int kv = kv_of(b), kb = kb_of(b);
       if (splits > 0) {
         for (int q = 0; q < parts; ++q) {
-          const int t0 = min(q * per_seg * ATT_TILE, kv), t1 = min((q + 1) * per_seg * ATT_TILE, kv);
-          units[u0 + q] = make_int4(b, t0, t1, parts > 1 ? sl0 + q : -1);
+          const int t0 = min(kb + q * per_seg * ATT_TILE, kv), t1 = min(kb + (q + 1) * per_seg * ATT_TILE, kv);
+          units[u0 + q] = make_int4(b, t0, t1, slotted ? sl0 + q : -1);
         }
       } else {
         // CTAs after the previous row's last one and up to this row's first
@@ -270,8 +291,8 @@ __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const i
           const int w = w0 + q;
           if (q > 0) work[w] = u0 + q;
           const int g0 = max(cum, w * per), g1 = min(cum + tiles, (w + 1) * per);
-          const int t0 = min((g0 - cum) * ATT_TILE, kv), t1 = min((g1 - cum) * ATT_TILE, kv);
-          units[u0 + q] = make_int4(b, t0, t1, parts > 1 ? sl0 + q : -1);
+          const int t0 = min(kb + (g0 - cum) * ATT_TILE, kv), t1 = min(kb + (g1 - cum) * ATT_TILE, kv);
+          units[u0 + q] = make_int4(b, t0, t1, slotted ? sl0 + q : -1);
         }
       }
     }
@@ -730,11 +751,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 // together, so a thread pays the L2 latency about once per four parts; CS
 // > 1 spreads rows of few sequences (long contexts) over more blocks.
 constexpr int COMBINE_THREADS = 256, COMBINE_HEADS = 8;
+// With o_f32 (partial decode) every row is written, in fp32: rows of one
+// segment are copied, rows with an empty range get o = 0 and lse = -inf.
 template <int CS>
 __global__ void __launch_bounds__(COMBINE_THREADS)
     mla_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                        const int4* __restrict__ row_info, int n_h, __nv_bfloat16* __restrict__ o_lat,
-                       float* __restrict__ lse) {
+                       float* __restrict__ lse, float* __restrict__ o_f32, const int32_t* __restrict__ kv_begin,
+                       const int32_t* __restrict__ kv_len) {
   constexpr int CPT = 16 / CS;  // columns per thread
   pdl_trigger();
   pdl_wait();
@@ -744,7 +768,15 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
   const int c0 = blockIdx.y * (ATT_DC / CS) + (threadIdx.x & 31) * CPT;
   const int4 info = row_info[r];
   const int n_parts = info.y, slot0 = info.z;
-  if (n_parts <= 1) return;  // written directly by its unit
+  if (n_parts <= (o_f32 ? 0 : 1)) return;  // written directly by its unit
+  if (o_f32 && kv_len[r] <= kv_begin[r]) {
+    // an empty range: no rows, no weight
+    float4* dst = reinterpret_cast<float4*>(o_f32 + ((long long)r * n_h + h) * ATT_DC + c0);
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q) dst[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (lse && c0 == 0) lse[(long long)r * n_h + h] = -INFINITY;
+    return;
+  }
   // online log-sum-exp over the parts' lse
   float mx = -INFINITY, tot = 0.f;
   for (int s = 0; s < n_parts; ++s) {
@@ -772,11 +804,98 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
       acc[4 * q + 3] += wgt * x[q].w;
     }
   }
-  uint2* dst = reinterpret_cast<uint2*>(o_lat + ((long long)r * n_h + h) * ATT_DC + c0);
+  if (o_f32) {
+    float4* dst = reinterpret_cast<float4*>(o_f32 + ((long long)r * n_h + h) * ATT_DC + c0);
 #pragma unroll
-  for (int q = 0; q < CPT / 4; ++q)
-    dst[q] = make_uint2(pack_bf16(acc[4 * q], acc[4 * q + 1]), pack_bf16(acc[4 * q + 2], acc[4 * q + 3]));
+    for (int q = 0; q < CPT / 4; ++q) dst[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+  } else {
+    uint2* dst = reinterpret_cast<uint2*>(o_lat + ((long long)r * n_h + h) * ATT_DC + c0);
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q)
+      dst[q] = make_uint2(pack_bf16(acc[4 * q], acc[4 * q + 1]), pack_bf16(acc[4 * q + 2], acc[4 * q + 3]));
+  }
   if (lse && c0 == 0) lse[(long long)r * n_h + h] = lse_all;
+}
+
+// Context-parallel merge of R ranks' partials of the same rows:
+// lse = log sum_r e^{lse_r}, o = sum_r e^{lse_r - lse} o_r.  A rank whose range
+// was empty contributes lse = -inf (weight 0).  Same block layout as the
+// combine (rows x 8 heads x column share).
+template <int CS>
+__global__ void __launch_bounds__(COMBINE_THREADS)
+    mla_lse_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int R, int rows,
+                         int n_h, __nv_bfloat16* __restrict__ o_bf16, float* __restrict__ o_f32,
+                         float* __restrict__ lse) {
+  constexpr int CPT = 16 / CS;
+  pdl_trigger();
+  pdl_wait();
+  const int groups = n_h / COMBINE_HEADS;
+  const int r = blockIdx.x / groups;
+  const int h = (blockIdx.x % groups) * COMBINE_HEADS + threadIdx.x / 32;
+  const int c0 = blockIdx.y * (ATT_DC / CS) + (threadIdx.x & 31) * CPT;
+  const long long stride = (long long)rows * n_h;  // one rank's lse block
+  float mx = -INFINITY;
+  for (int k = 0; k < R; ++k) mx = fmaxf(mx, lse_parts[k * stride + (long long)r * n_h + h]);
+  float tot = 0.f;
+  for (int k = 0; k < R; ++k) {
+    const float l = lse_parts[k * stride + (long long)r * n_h + h];
+    tot += l == -INFINITY ? 0.f : expf(l - mx);
+  }
+  const float lse_all = mx + logf(tot);
+  float acc[CPT];
+#pragma unroll
+  for (int e = 0; e < CPT; ++e) acc[e] = 0.f;
+  for (int k = 0; k < R; ++k) {
+    const float l = lse_parts[k * stride + (long long)r * n_h + h];
+    if (l == -INFINITY) continue;
+    const float wgt = expf(l - lse_all);
+    const float4* src = reinterpret_cast<const float4*>(o_parts + (k * stride + (long long)r * n_h + h) * ATT_DC + c0);
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q) {
+      const float4 x = src[q];
+      acc[4 * q] += wgt * x.x;
+      acc[4 * q + 1] += wgt * x.y;
+      acc[4 * q + 2] += wgt * x.z;
+      acc[4 * q + 3] += wgt * x.w;
+    }
+  }
+  const long long ob = ((long long)r * n_h + h) * ATT_DC + c0;
+  if (o_f32) {
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q)
+      reinterpret_cast<float4*>(o_f32 + ob)[q] = make_float4(acc[4 * q], acc[4 * q + 1], acc[4 * q + 2], acc[4 * q + 3]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < CPT / 4; ++q)
+      reinterpret_cast<uint2*>(o_bf16 + ob)[q] =
+          make_uint2(pack_bf16(acc[4 * q], acc[4 * q + 1]), pack_bf16(acc[4 * q + 2], acc[4 * q + 3]));
+  }
+  if (lse && c0 == 0) lse[(long long)r * n_h + h] = lse_all;
+}
+
+// The same merge for any d_c (fp32 layers): one block per (row, head).
+__global__ void mla_lse_merge_any_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int R,
+                                         int rows, int n_h, int d_c, float* __restrict__ o_f32,
+                                         float* __restrict__ lse) {
+  const int r = blockIdx.x / n_h, h = blockIdx.x % n_h;
+  const long long stride = (long long)rows * n_h;
+  float mx = -INFINITY;
+  for (int k = 0; k < R; ++k) mx = fmaxf(mx, lse_parts[k * stride + (long long)r * n_h + h]);
+  float tot = 0.f;
+  for (int k = 0; k < R; ++k) {
+    const float l = lse_parts[k * stride + (long long)r * n_h + h];
+    tot += l == -INFINITY ? 0.f : expf(l - mx);
+  }
+  const float lse_all = mx + logf(tot);
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
+    float acc = 0.f;
+    for (int k = 0; k < R; ++k) {
+      const float l = lse_parts[k * stride + (long long)r * n_h + h];
+      if (l != -INFINITY) acc += expf(l - lse_all) * o_parts[(k * stride + (long long)r * n_h + h) * d_c + c];
+    }
+    o_f32[((long long)r * n_h + h) * d_c + c] = acc;
+  }
+  if (lse && threadIdx.x == 0) lse[(long long)r * n_h + h] = lse_all;
 }
 
 }  // namespace mla

@@ -333,7 +333,9 @@ inline int attn_groups(const mla_layer_desc* D) { return use_pair_kernel(D) ? 1 
 inline int attn_wave_workers(const mla_layer_desc* D) {
   return std::max(1, use_pair_kernel(D) ? num_sms() / 2 : num_sms() / attn_groups(D));
 }
-inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int requested, int workers = 0) {
+// force: every segment gets a partial slot (partial decode: all rows go out in fp32 through the combine)
+inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int requested, int workers = 0,
+                          bool force = false) {
   AttnPlan p{};
   const int max_tiles = std::max(1, (max_len + ATT_TILE - 1) / ATT_TILE);
   if (requested == 1) {
@@ -347,7 +349,7 @@ inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int re
     p.splits = std::min(requested, max_tiles);
     p.max_units = rows * p.splits;
     p.workers = p.max_units;
-    p.max_slots = p.splits > 1 ? p.max_units : 0;
+    p.max_slots = (p.splits > 1 || force) ? p.max_units : 0;
     return p;
   }
   p.splits = 0;
@@ -355,7 +357,7 @@ inline AttnPlan plan_attn(const mla_layer_desc* D, int rows, int max_len, int re
   // each range boundary cuts at most one row: segments <= rows + workers - 1,
   // and the segments of cut rows number at most 2 * (workers - 1)
   p.max_units = rows + p.workers;
-  p.max_slots = std::min(p.max_units, 2 * p.workers);
+  p.max_slots = force ? p.max_units : std::min(p.max_units, 2 * p.workers);
   return p;
 }
 // Workspace carve of one plan: segment list, row table, CTA table, partials.
@@ -398,6 +400,7 @@ static size_t tc_workspace_size(const mla_layer_desc* D, int T, int B, int max_k
     const int max_len = (max_kv_len + 63) / 64 * 64;
     // the automatic plan, or any explicit split count up to 16
     w = std::max(w, ws_attn(D, B, plan_attn(D, B, max_len, 0)));
+    w = std::max(w, ws_attn(D, B, plan_attn(D, B, max_len, 0, 0, /*force=*/true)));  // partial decode
     w = std::max(w, ws_attn(D, B, plan_attn(D, B, max_len, 16)));
   }
   return w + 256;
@@ -617,6 +620,25 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
   return MLA_OK;
 }
 
+// Merge R partials [R][rows][n_h][d_c] (+ lse [R][rows][n_h]) into o (desc dtype) and lse.
+static mla_status_t tc_lse_merge(const mla_layer_desc* D, const float* o_parts, const float* lse_parts, int R, int rows,
+                                 void* o, float* lse, cudaStream_t st) {
+  if (D->dtype == MLA_F32 || D->d_c != ATT_DC || D->n_h % COMBINE_HEADS != 0) {
+    MLA_COUNT_LAUNCH();
+    mla_lse_merge_any_kernel<<<rows * D->n_h, 128, 0, st>>>(o_parts, lse_parts, R, rows, D->n_h, D->d_c, (float*)o,
+                                                             lse);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  }
+  if (!aligned16(o_parts) || !aligned16(o)) return MLA_ERR_INVALID_ARG;
+  const int blocks = rows * (D->n_h / COMBINE_HEADS);
+  const int cs = blocks >= 2 * num_sms() ? 1 : blocks >= num_sms() ? 2 : 4;
+  auto kfn = cs == 1 ? mla_lse_merge_kernel<1> : cs == 2 ? mla_lse_merge_kernel<2> : mla_lse_merge_kernel<4>;
+  return launch_pdl(kfn, dim3(blocks, cs), dim3(COMBINE_THREADS), 0, st, 1, o_parts, lse_parts, R, rows, D->n_h,
+                    (__nv_bfloat16*)o, (float*)nullptr, lse) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
 template <int H>
 static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, const CUtensorMap& mc, const AttnArgs& a,
                                dim3 grid, cudaStream_t st) {
@@ -626,15 +648,20 @@ static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, con
   return launch_pdl(kfn, grid, dim3(ATT_THREADS), smem, st, 1, mq, mr, mc, a);
 }
 
+// kv_begin (partial decode): rows [kv_begin[b], kv_len[b]) only, every row
+// written in fp32 to o_f32 (o_lat unused) with its lse.
 static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
                                  const mla_paged_cache* cache, const int32_t* kv_len, const int32_t* q_start,
                                  int q_per_seq, int rows, void* ws, size_t ws_bytes, int num_splits, void* o_lat,
-                                 float* lse, cudaStream_t st, int workers = 0) {
-  if (!aligned16(q_lat) || !aligned16(q_rope) || !aligned16(cache->pool) || !aligned16(o_lat))
+                                 float* lse, cudaStream_t st, int workers = 0, const int32_t* kv_begin = nullptr,
+                                 float* o_f32 = nullptr) {
+  if (!aligned16(q_lat) || !aligned16(q_rope) || !aligned16(cache->pool) || !aligned16(kv_begin ? o_f32 : o_lat))
     return MLA_ERR_INVALID_ARG;
   const int H = heads_per_cta(D);
   const int max_len = cache->max_blocks * 64;
-  const AttnPlan p = plan_attn(D, rows, max_len, kv_len ? num_splits : 1, workers);
+  const bool partial = kv_begin != nullptr;
+  const AttnPlan p = plan_attn(D, rows, max_len, kv_len ? (partial && num_splits == 1 ? 0 : num_splits) : 1, workers,
+                               partial);
   Carver cv = carve(ws, ws_bytes);
   AttnWs aw{};
   if (p.use_plan && (!ws || !carve_attn(cv, D, rows, p, &aw))) return MLA_ERR_CAPACITY;
@@ -642,7 +669,7 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
     const int threads = std::min(1024, std::max(32, (rows + 31) / 32 * 32));
     if (launch_pdl(mla_attn_plan_kernel, dim3(1), dim3(threads), 0, st, 1, kv_len, q_start, q_per_seq, rows,
                    max_len, p.workers, p.splits, p.max_units, p.max_slots, aw.units, aw.row_info, aw.work,
-                   aw.n_units) != cudaSuccess)
+                   aw.n_units, kv_begin, partial ? 1 : 0) != cudaSuccess)
       return MLA_ERR_CUDA;
   }
   const bool pair = use_pair_kernel(D);
@@ -662,6 +689,7 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   a.table = cache->block_table;
   a.pool = (const uint8_t*)cache->pool;
   a.kv_len = kv_len;
+  a.kv_begin = kv_begin;
   a.q_start = q_start;
   a.o_lat = (__nv_bfloat16*)o_lat;
   a.lse = lse;
@@ -691,7 +719,8 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
     const dim3 grid(blocks, cs);
     auto kfn = cs == 1 ? mla_combine_kernel<1> : cs == 2 ? mla_combine_kernel<2> : mla_combine_kernel<4>;
     if (launch_pdl(kfn, grid, dim3(COMBINE_THREADS), 0, st, 1, (const float*)aw.o_part, (const float*)aw.lse_part,
-                   (const int4*)aw.row_info, D->n_h, (__nv_bfloat16*)o_lat, lse) != cudaSuccess)
+                   (const int4*)aw.row_info, D->n_h, (__nv_bfloat16*)o_lat, lse, o_f32, kv_begin, kv_len) !=
+        cudaSuccess)
       return MLA_ERR_CUDA;
   }
   return MLA_OK;

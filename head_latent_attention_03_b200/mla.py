@@ -69,6 +69,12 @@ _SIGS = {
                                         ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_void_p]),
+    "mla_decode_attn_partial": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p]),
+    "mla_lse_merge": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "mla_out_proj": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                     ctypes.c_void_p]),
@@ -166,6 +172,23 @@ def decode_attn_noalloc(desc, q_lat, q_rope, cache: PagedCache, kv_len, o_lat, l
     _check("mla_decode_attn_noalloc", lib().mla_decode_attn_noalloc(
         ctypes.byref(desc), _ptr(q_lat), _ptr(q_rope), ctypes.byref(cache), _ptr(kv_len), kv_len.shape[0],
         num_splits, _ptr(o_lat), _ptr(lse), _stream(stream)))
+
+
+def decode_attn_partial(desc, q_lat, q_rope, cache: PagedCache, kv_begin, kv_end, ws, o_part, lse_part,
+                        stream=None):
+    """Attention over rows [kv_begin, kv_end) of each sequence: fp32 o_part
+    (normalised within the range) and lse_part, for a context-parallel merge."""
+    _check("mla_decode_attn_partial", lib().mla_decode_attn_partial(
+        ctypes.byref(desc), _ptr(q_lat), _ptr(q_rope), ctypes.byref(cache), _ptr(kv_begin), _ptr(kv_end),
+        kv_end.shape[0], _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _ptr(o_part),
+        _ptr(lse_part), _stream(stream)))
+
+
+def lse_merge(desc, o_parts, lse_parts, o_lat, lse=None, stream=None):
+    """Merge R partials o_parts [R, B, n_h, d_c], lse_parts [R, B, n_h] into o_lat, lse."""
+    _check("mla_lse_merge", lib().mla_lse_merge(
+        ctypes.byref(desc), _ptr(o_parts), _ptr(lse_parts), o_parts.shape[0], o_parts.shape[1], _ptr(o_lat),
+        _ptr(lse), _stream(stream)))
 
 
 def prefill_attn(desc, q_lat, q_rope, cache: PagedCache, q_start, q_per_seq, ws, o_lat, lse=None, stream=None):

@@ -191,6 +191,35 @@ mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* desc, const void* q_l
                                      const mla_paged_cache* cache, const int32_t* kv_len, int B, int num_splits,
                                      void* o_lat, float* lse, void* stream);
 
+/* Context parallelism for long decodes (the pages' 128K-context setting, DeepSeek-V2
+ * explainer section 3.1.3): the pages of one sequence are spread over R GPUs,
+ * each attends to the rows it holds, and the ranks' results are merged by
+ * log-sum-exp after one exchange of n_h * (d_c + 1) floats per sequence.
+ *
+ * mla_decode_attn_partial: decode attention over rows [kv_begin[b], kv_end[b])
+ * of each sequence only (the rows this GPU holds; pages outside the range are
+ * never read, so block_table may leave them unset).
+ *   kv_begin [B] int32   a multiple of 128 (0 <= kv_begin <= kv_end); a bad
+ *                        value empties the row and sets MLA_ERR_CAPACITY in
+ *                        the device error word
+ *   kv_end   [B] int32   <= max_blocks * block_size; kv_end == kv_begin is an
+ *                        empty range: o_part = 0, lse_part = -inf
+ *   o_part   [B, n_h, d_c] float  out: softmax-weighted sum of c^KV over the range
+ *   lse_part [B, n_h] float       out: log sum over the range of exp(s_j)
+ * Workspace: mla_workspace_size(desc, 0, B, max kv_end).  bf16 layers only
+ * (MLA_ERR_UNSUPPORTED for MLA_F32).
+ *
+ * mla_lse_merge: merges R partials of the same B rows,
+ *   lse = log sum_r exp(lse_r),  o = sum_r exp(lse_r - lse) o_r   (lse_r = -inf: weight 0)
+ *   o_parts [R, B, n_h, d_c] float, lse_parts [R, B, n_h] float (rank-major, as an
+ *   all-gather lays them out); o_lat [B, n_h, d_c] desc dtype, lse [B, n_h]
+ *   float (may be NULL). */
+mla_status_t mla_decode_attn_partial(const mla_layer_desc* desc, const void* q_lat, const void* q_rope,
+                                     const mla_paged_cache* cache, const int32_t* kv_begin, const int32_t* kv_end,
+                                     int B, void* ws, size_t ws_bytes, float* o_part, float* lse_part, void* stream);
+mla_status_t mla_lse_merge(const mla_layer_desc* desc, const float* o_parts, const float* lse_parts, int R, int B,
+                           void* o_lat, float* lse, void* stream);
+
 /* Causal attention of a chunk of q_per_seq new queries per sequence (chunked
  * prefill, after mla_compress_append of the chunk).  Query q of sequence b
  * sits at position q_start[b] + q and attends rows 0 .. q_start[b] + q.

@@ -214,6 +214,19 @@ def attend_absorbed(D, W, q_lat: np.ndarray, q_r: np.ndarray, rows: np.ndarray):
     return o_lat, lse, u
 
 
+def merge_partials(o_parts: Sequence[np.ndarray], lse_parts: Sequence[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:
+    """Attention over the union of disjoint row sets from the attentions over
+    each set: with Z_r = sum over set r of e^{z_j} = e^{lse_r}, the softmax over
+    the union weighs set r by Z_r / sum Z; lse = log sum Z.  An empty set has
+    lse = -inf and weight 0.  Arrays [..., d] and [...] per part."""
+    lse = np.stack([np.asarray(l, dtype=F64) for l in lse_parts])
+    m = np.max(lse, axis=0)
+    w = np.exp(lse - m)
+    tot = np.sum(w, axis=0)
+    out = sum(w[r][..., None] * np.asarray(o_parts[r], dtype=F64) for r in range(len(o_parts))) / tot[..., None]
+    return out, m + np.log(tot)
+
+
 def out_project(D, W, o_lat: np.ndarray) -> np.ndarray:
     """u = W^O [W^UV_1 o_lat_1; ...; W^UV_nh o_lat_nh] (eq 8 with W^UV absorbed)."""
     w_uv = W["w_uv"].astype(F64).reshape(D.n_h, D.d_h, D.d_c)

@@ -253,3 +253,64 @@ def test_prefill_sampled(b, qs):
         assert_bf16(np32(st.o_lat)[b * n + q], outs[q]["o_lat"], f"o_lat q={q}")
         assert np.max(np.abs(np32(st.lse)[b * n + q] - outs[q]["lse"])) < 2e-2
         assert_bf16(np32(st.u)[b * n + q], outs[q]["u"], f"u q={q}")
+
+
+# ----------------------------------------------------------------------------
+# context parallelism: each rank's partial over its shard of the rows (the
+# ranks run one after another on this GPU; each reads only its rows), merged
+# by log-sum-exp
+# ----------------------------------------------------------------------------
+def _cp_merge(layer, st, batch, world):
+    from head_latent_attention_03_b200.context_parallel import shard_ranges
+    D = batch.workload.dims
+    B = len(batch.prior_len)
+    ranges = shard_ranges(batch.prior_len + 1, world)
+    o_parts = torch.empty((world, B, D.n_h, D.d_c), dtype=torch.float32, device="cuda")
+    l_parts = torch.empty((world, B, D.n_h), dtype=torch.float32, device="cuda")
+    cache = layer.cache(st)
+    for r in range(world):
+        kb = torch.from_numpy(ranges[r, :, 0].copy()).cuda()
+        ke = torch.from_numpy(ranges[r, :, 1].copy()).cuda()
+        mla.decode_attn_partial(layer.desc, st.q_lat, st.q_rope, cache, kb, ke, st.ws, o_parts[r], l_parts[r])
+    o = torch.empty_like(st.o_lat)
+    l = torch.empty_like(st.lse)
+    mla.lse_merge(layer.desc, o_parts, l_parts, o, l)
+    torch.cuda.synchronize()
+    assert mla.get_last_error() == 0
+    return ranges, o_parts, l_parts, o, l
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_merge(world):
+    w = dataclasses.replace(I.WORKLOADS["v2"], name="v2_cp", batch=3, prior="list:1000,3000,129")
+    batch = I.gen_batch(w)
+    layer, st = run_gpu(w, batch)
+    D, W = w.dims, weights_for(w)
+    ranges, o_parts, l_parts, o, l = _cp_merge(layer, st, batch, world)
+    # one rank's partial against the oracle over that rank's rows
+    ref = O.decode_batch(batch, W, absorbed=True)
+    r = world - 1
+    for b in range(3):
+        lo, hi = ranges[r, b]
+        rows = O.gather_rows(batch.pool, batch.block_table[b], int(batch.prior_len[b]), D.block_size)
+        rows = np.concatenate([rows, ref[b]["row"][None]], axis=0)
+        if hi > lo:
+            po, pl, _ = O.attend_absorbed(D, W, ref[b]["q_lat"], ref[b]["q_r"], rows[lo:hi])
+            assert_bf16(np32(o_parts[r, b]), po, f"partial o rank {r} seq {b}")
+            assert np.max(np.abs(np32(l_parts[r, b]) - pl)) < 2e-2
+        else:
+            assert np.all(np32(o_parts[r, b]) == 0) and np.all(np.isneginf(np32(l_parts[r, b])))
+    # the merge against the oracle over all rows and against mla_decode_attn
+    assert_bf16(np32(o), np.stack([x["o_lat"] for x in ref]), "merged o_lat")
+    assert np.max(np.abs(np32(l) - np.stack([x["lse"] for x in ref]))) < 2e-2
+    assert_bf16(np32(o), np32(st.o_lat), "merged vs one-GPU decode")
+
+
+def test_context_parallel_long_context():
+    # 4 x 131073 rows over 4 ranks: the merged result is the one-GPU decode
+    w = I.WORKLOADS["long"]
+    batch = I.gen_batch(w)
+    layer, st = run_gpu(w, batch)
+    _, _, _, o, l = _cp_merge(layer, st, batch, 4)
+    assert_bf16(np32(o), np32(st.o_lat), "merged vs one-GPU decode")
+    assert np.max(np.abs(np32(l) - np32(st.lse))) < 2e-2

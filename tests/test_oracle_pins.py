@@ -435,3 +435,30 @@ def test_latent_norm_epsilon_closed_form():
     m = float(np.mean(raw * raw))
     y = O.compress_kv(D, W, h, 0)[:D.d_c]
     assert abs(float(np.mean(y * y)) - m / (m + D.norm_eps)) < 1e-13
+
+
+# Context parallelism (the attention over a sequence's rows split between
+# ranks): the softmax over a union of disjoint row sets is the sets' softmaxes
+# weighted by their partition sums, so the merged partial attentions are the
+# attention over all rows (1e-12), an empty set included.
+def test_merged_partials_equal_attention_over_all_rows():
+    rng = np.random.default_rng(41)
+    D = SMALL[1]
+    W = _rand_weights(D, rng)
+    rows = rng.standard_normal((70, D.row)) * 1.5
+    q_lat = rng.standard_normal((D.n_h, D.d_c))
+    q_r = rng.standard_normal((D.n_h, D.d_hr))
+    full_o, full_lse, _ = O.attend_absorbed(D, W, q_lat, q_r, rows)
+    cuts = [(0, 0), (0, 23), (23, 64), (64, 70)]  # the first rank holds no rows
+    parts_o, parts_l = [], []
+    for a, b in cuts:
+        if a == b:
+            parts_o.append(np.zeros((D.n_h, D.d_c)))
+            parts_l.append(np.full(D.n_h, -np.inf))
+        else:
+            o, l, _ = O.attend_absorbed(D, W, q_lat, q_r, rows[a:b])
+            parts_o.append(o)
+            parts_l.append(l)
+    o, lse = O.merge_partials(parts_o, parts_l)
+    assert np.max(np.abs(o - full_o)) <= 1e-12 * np.max(np.abs(full_o))
+    assert np.max(np.abs(lse - full_lse)) <= 1e-12 * np.max(np.abs(full_lse))

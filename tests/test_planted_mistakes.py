@@ -53,6 +53,10 @@ MUTATIONS = {
     # query latent left un-normalised
     "norm_query_skipped": ("c_q = latent_norm(D, W, W[\"w_dq\"].astype(F64) @ h, \"q\") if D.d_cq else h",
                            "c_q = W[\"w_dq\"].astype(F64) @ h if D.d_cq else h"),
+    # merge of partial attentions without the normaliser
+    "merge_unnormalised": ("/ tot[..., None]", ""),
+    # merge weighing the parts equally
+    "merge_equal_weights": ("w = np.exp(lse - m)", "w = np.ones_like(lse)"),
     # W^O applied before W^UV's head split is undone
     "out_proj_heads": ("o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64))",
                        "o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64)[::-1])"),
