@@ -752,6 +752,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 11, 0);
+  // A role of this CTA gave up a wait: its peer's roles may be waiting for
+  // this CTA's signals, so raise the peer's abort flag too (their waits poll
+  // it) rather than let each of them run into its own time limit.
+  if (threadIdx.x == 0 && *abort_flag)
+    st_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u), 1u);
   cluster_sync_all();  // the peer's MMAs, TMA signals and arrives are done
   if (warp == 1) tmem_dealloc_pair(tmem, C::TMEM_COLS);
 }

@@ -189,6 +189,31 @@ def test_bad_page_id_reports_capacity_error():
     assert mla.get_last_error() == 0  # cleared
 
 
+@pytest.mark.parametrize("w", [LITE_SMALL, V2_SMALL], ids=lambda w: w.name)
+def test_out_of_range_kv_len_reports_capacity_error(w):
+    # kv_len beyond the page table (max_blocks * 64) and kv_len = 0: the plan
+    # clamps the rows it deals out and the kernels skip the segment, so no
+    # page outside the table is read; the call reports MLA_ERR_CAPACITY
+    batch = I.gen_batch(w)
+    layer = MLALayer(w.dims, weights_for(w))
+    st = layer.upload(batch)
+    layer.compress_append(st)
+    layer.absorb_q(st)
+    torch.cuda.synchronize()
+    assert mla.get_last_error() == 0
+    for bad in (st.table.shape[1] * 64 + 5, 0):
+        kv = st.kv_len.clone()
+        kv[1] = bad
+        mla.decode_attn(layer.desc, st.q_lat, st.q_rope, layer.cache(st), kv, st.ws, st.o_lat, st.lse)
+        assert mla.get_last_error() == 3  # MLA_ERR_CAPACITY, no fault
+        assert mla.get_last_error() == 0  # cleared
+    # the next valid call is unaffected
+    layer.attend(st)
+    layer.out_proj(st)
+    torch.cuda.synchronize()
+    assert mla.get_last_error() == 0
+
+
 # ----------------------------------------------------------------------------
 # full-size workloads, in the launch configuration bench.py times; the oracle
 # checks a sample of sequences
