@@ -270,6 +270,43 @@ mla_status_t mla_lse_merge(const mla_layer_desc* D, const float* o_parts, const 
   return tc_lse_merge(D, o_parts, lse_parts, R, B, o_lat, lse, as_stream(stream));
 }
 
+size_t mla_prefill_unabsorbed_workspace_size(const mla_layer_desc* D, int num_blocks, int B, int max_blocks) {
+  if (!desc_valid(D) || num_blocks < 0 || B < 0 || max_blocks < 0) return 0;
+  return ws_prefill_unabsorbed(D, num_blocks, B, max_blocks);
+}
+
+mla_status_t mla_queries(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos, int T,
+                         void* q_c, void* q_rope, void* ws, size_t ws_bytes, void* stream) {
+  if (!desc_valid(D) || !w || !w->w_uq || !w->w_qr || (D->d_cq && !w->w_dq) || !h || !pos || T < 0 || !q_c ||
+      !q_rope || (D->latent_norm && D->d_cq && !w->g_q))
+    return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (D->dtype != MLA_BF16 || !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_absorb_q(D, w, h, pos, T, nullptr, q_rope, ws, ws_bytes, as_stream(stream), q_c);
+}
+
+mla_status_t mla_prefill_attn_unabsorbed(const mla_layer_desc* D, const mla_weights* w, const void* q_c,
+                                         const void* q_rope, const mla_paged_cache* cache, const int32_t* q_start,
+                                         int q_per_seq, int B, void* ws, size_t ws_bytes, void* o, float* lse,
+                                         void* stream) {
+  if (!desc_valid(D) || !w || !w->w_uk || !w->w_uv || !q_c || !q_rope || !cache_valid(cache) || !q_start ||
+      q_per_seq <= 0 || B < 0 || !o)
+    return MLA_ERR_INVALID_ARG;
+  if (B == 0) return MLA_OK;
+  if ((long long)B * q_per_seq > (1 << 30)) return MLA_ERR_UNSUPPORTED;
+  if (D->dtype != MLA_BF16 || !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_prefill_unabsorbed(D, w, q_c, q_rope, cache, q_start, q_per_seq, B, ws, ws_bytes, o, lse,
+                               as_stream(stream));
+}
+
+mla_status_t mla_out_proj_unabsorbed(const mla_layer_desc* D, const mla_weights* w, const void* o, int T, float* u,
+                                     void* stream) {
+  if (!desc_valid(D) || !w || !w->w_o || !o || T < 0 || !u) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (D->dtype != MLA_BF16 || !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_out_proj(D, w, o, T, u, nullptr, 0, as_stream(stream), /*from_o=*/true);
+}
+
 mla_status_t mla_prefill_attn(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
                               const mla_paged_cache* cache, const int32_t* q_start, int q_per_seq, int B, void* ws,
                               size_t ws_bytes, void* o_lat, float* lse, void* stream) {

@@ -70,6 +70,9 @@ struct GemmArgs {
   int T;               // tokens
   int a_z_rows;        // per-batch row offset into A (K-major: output rows; MN-major: K rows)
   int b_z_cols;        // per-batch column offset into X
+  // optional: token tile nt reads (and writes) rows b_tile_row[nt] .. + TN of
+  // X and Y (cache pages scattered over the pool); nullptr: rows nt * TN ..
+  const int32_t* b_tile_row;
   GemmEpi e;
 };
 
@@ -179,7 +182,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
   const int mt = blockIdx.x / S, ks = blockIdx.x % S;  // ks = rank in the cluster
   const int nt = blockIdx.y, z = blockIdx.z;
   const int kc0 = ks * g.k_chunks_split;
-  const int nk = max(0, min(g.k_chunks_split, g.k_chunks - kc0));
+  int nk = max(0, min(g.k_chunks_split, g.k_chunks - kc0));
+  if (g.b_tile_row) {
+    // a page-indexed token tile with row -1 (past its sequence) does nothing
+    pdl_wait();
+    if (g.b_tile_row[nt] < 0) nk = 0;
+  }
   const bool seg1 = mt >= g.m_tiles0;
   const CUtensorMap* mA = seg1 ? &mA1 : &mA0;
   const int m_row0 = (seg1 ? mt - g.m_tiles0 : mt) * GEMM_BM;  // first row inside the segment
@@ -217,8 +225,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
           tma_load_2d(sa + 8192, mA, &full[i % C::NST], m_row0 + 64, z * g.a_z_rows + kc * GEMM_BK);
         }
       };
+      int b_row0 = nt * TN;  // a page-indexed tile's row is read after pdl_wait below
       auto load_b = [&](int i, uint8_t* sb) {
-        tma_load_3d(sb, &mB, &full[i % C::NST], 0, nt * TN, z * g.b_z_cols / GEMM_BK + kc0 + i * KC);
+        tma_load_3d(sb, &mB, &full[i % C::NST], 0, b_row0, z * g.b_z_cols / GEMM_BK + kc0 + i * KC);
       };
       // While the previous kernel finishes, pull this CTA's first weight
       // tiles into L2; every load into shared memory waits for it.
@@ -233,6 +242,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
         }
       }
       pdl_wait();
+      if (g.b_tile_row) b_row0 = g.b_tile_row[nt];
       for (int i = 0; i < pre; ++i) {
         mbar_expect_tx(&full[i], C::STAGE);
         load_a(i, smem + i * C::STAGE);
@@ -328,9 +338,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
         const int e = e0 + q * GEMM_THREADS;
         if (e >= n_el) continue;
         const int t_loc = e / n_pairs, rr = r0 + 2 * (e % n_pairs);
-        const int t = nt * TN + t_loc;
+        const int t = (g.b_tile_row ? g.b_tile_row[nt] : nt * TN) + t_loc;
         const int n_in_seg = m_row0 + rr;
-        if (t >= g.T || n_in_seg >= n_seg) continue;
+        if (t >= g.T || n_in_seg >= n_seg || (g.b_tile_row && g.b_tile_row[nt] < 0)) continue;
         float2 v = part[q][0];
 #pragma unroll
         for (int sr = 1; sr < SMAX; ++sr)

@@ -21,6 +21,7 @@
 #include "tc_attn.cuh"
 #include "tc_attn2.cuh"
 #include "tc_gemm.cuh"
+#include "tc_prefill.cuh"
 
 namespace mla {
 
@@ -224,6 +225,8 @@ struct GemmCall {
   const void* x;
   long long x_rows, x_row_elems;  // X map: x_rows rows of x_row_elems
   int K, T, Z, a_z_rows, b_z_cols;
+  const int32_t* b_tile_row;  // optional page-indexed token tiles (see GemmArgs)
+  int n_tiles_override;       // with b_tile_row: the number of token tiles
 };
 
 inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan& p, cudaStream_t st) {
@@ -251,9 +254,10 @@ inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan
   g.T = c.T;
   g.a_z_rows = c.a_z_rows;
   g.b_z_cols = c.b_z_cols;
+  g.b_tile_row = c.b_tile_row;
   g.e = e;
   const int m_tiles = g.m_tiles0 + (c.a1 ? (c.rows1 + GEMM_BM - 1) / GEMM_BM : 0);
-  dim3 grid(m_tiles * p.splits, p.n_tiles, c.Z);
+  dim3 grid(m_tiles * p.splits, c.b_tile_row ? c.n_tiles_override : p.n_tiles, c.Z);
   cudaError_t err;
   if (c.a_mn)
     err = p.deep ? launch_gemm_tn<true, true>(p.tn, A0, A1, B, g, grid, st)
@@ -261,6 +265,32 @@ inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan
   else
     err = p.deep ? launch_gemm_tn<false, true>(p.tn, A0, A1, B, g, grid, st)
                  : launch_gemm_tn<false, false>(p.tn, A0, A1, B, g, grid, st);
+  return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// A GEMM whose token tiles are cache pages (c.b_tile_row): X rows are
+// x_row_bytes apart (the pool's [c^KV | k^R] rows), the plan is the caller's.
+inline mla_status_t run_gemm_paged(const GemmCall& c, const GemmEpi& e, const GemmPlan& p, uint64_t x_row_bytes,
+                                   cudaStream_t st) {
+  CUtensorMap A0, A1, B;
+  bool ok = map_rows_chunks(&A0, c.a0, (uint64_t)c.K, (uint64_t)c.rows0, (uint64_t)c.a_row_elems * 2, 128, 1);
+  ok = ok && map_rows_chunks(&A1, c.a1, (uint64_t)c.K, (uint64_t)c.rows1, (uint64_t)c.a_row_elems * 2, 128, 1);
+  ok = ok && map_rows_chunks(&B, c.x, (uint64_t)c.x_row_elems, (uint64_t)c.x_rows, x_row_bytes, 64, 1);
+  if (!ok) return MLA_ERR_CUDA;
+  GemmArgs g;
+  g.k_chunks = c.K / GEMM_BK;
+  g.k_chunks_split = p.kcs;
+  g.splits = 1;
+  g.m_tiles0 = (c.rows0 + GEMM_BM - 1) / GEMM_BM;
+  g.n_out0 = c.rows0;
+  g.n_out1 = c.rows1;
+  g.T = c.T;
+  g.a_z_rows = 0;
+  g.b_z_cols = 0;
+  g.b_tile_row = c.b_tile_row;
+  g.e = e;
+  const int m_tiles = g.m_tiles0 + (c.rows1 + GEMM_BM - 1) / GEMM_BM;
+  const cudaError_t err = launch_gemm_t<64, false, false>(A0, A1, B, g, dim3(m_tiles, p.n_tiles, 1), st);
   return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -473,8 +503,11 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
                                                                                                       : MLA_ERR_CUDA;
 }
 
+// q_c_out: write q^C [T, n_h, d_h] there (the un-absorbed prefill's queries);
+// q_lat may then be null (no W^UK absorption).
 static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos,
-                                int T, void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st) {
+                                int T, void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st,
+                                void* q_c_out = nullptr) {
   if (!aligned16(h) || !aligned16(w->w_uq) || !aligned16(w->w_qr) || !aligned16(w->w_uk) ||
       (D->d_cq && !aligned16(w->w_dq)) || !aligned16(q_lat) || !aligned16(q_rope) ||
       (D->d_cq && D->latent_norm && !aligned16(w->g_q)))
@@ -483,7 +516,8 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
   const int nq = D->n_h * D->d_h, nr = D->n_h * D->d_hr;
   const int q_in = D->d_cq ? D->d_cq : D->d;
   __nv_bfloat16* cq = D->d_cq ? (__nv_bfloat16*)cv.take((size_t)T * D->d_cq * 2) : nullptr;
-  __nv_bfloat16* qc = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
+  __nv_bfloat16* qc = q_c_out ? (__nv_bfloat16*)q_c_out : (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
+  if (q_c_out && !aligned16(q_c_out)) return MLA_ERR_INVALID_ARG;
   float* cq32 = D->d_cq && D->latent_norm ? (float*)cv.take((size_t)T * D->d_cq * 4) : nullptr;
   if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   mla_status_t s;
@@ -547,6 +581,7 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     e.q_rope = (__nv_bfloat16*)q_rope;
     if ((s = run_gemm(c, e, plan_q2(D, T), st)) != MLA_OK) return s;
   }
+  if (!q_lat) return MLA_OK;  // queries only (the un-absorbed prefill reads q^C)
   {  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major
     GemmCall c{};
     c.a0 = w->w_uk;
@@ -572,15 +607,16 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
   return MLA_OK;
 }
 
+// from_o: the input is o [T, n_h, d_h] itself (un-absorbed prefill): W^O only.
 static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, const void* o_lat, int T, float* u,
-                                void* ws, size_t ws_bytes, cudaStream_t st) {
+                                void* ws, size_t ws_bytes, cudaStream_t st, bool from_o = false) {
   if (!aligned16(o_lat) || !aligned16(w->w_uv) || !aligned16(w->w_o)) return MLA_ERR_INVALID_ARG;
   Carver cv = carve(ws, ws_bytes);
   const int nq = D->n_h * D->d_h;
-  __nv_bfloat16* o = (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
-  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  __nv_bfloat16* o = from_o ? (__nv_bfloat16*)o_lat : (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
+  if (!from_o && (!ws || !cv.ok())) return MLA_ERR_CAPACITY;
   mla_status_t s;
-  {  // o_i = W^UV_i o_lat_i  (eq 11 absorbed): per head, A = W^UV_i [d_h, d_c]
+  if (!from_o) {  // o_i = W^UV_i o_lat_i  (eq 11 absorbed): per head, A = W^UV_i [d_h, d_c]
     GemmCall c{};
     c.a0 = w->w_uv;
     c.rows0 = D->d_h;
@@ -635,6 +671,106 @@ static mla_status_t tc_lse_merge(const mla_layer_desc* D, const float* o_parts, 
   auto kfn = cs == 1 ? mla_lse_merge_kernel<1> : cs == 2 ? mla_lse_merge_kernel<2> : mla_lse_merge_kernel<4>;
   return launch_pdl(kfn, dim3(blocks, cs), dim3(COMBINE_THREADS), 0, st, 1, o_parts, lse_parts, R, rows, D->n_h,
                     (__nv_bfloat16*)o, (float*)nullptr, lse) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// un-absorbed chunked prefill (tc_prefill.cuh)
+// ---------------------------------------------------------------------------
+// rows[b * max_blocks + j]: first pool row of page j of sequence b, or -1 past
+// the sequence's end after the chunk (q_start[b] + q_per_seq rows)
+__global__ void mla_page_rows_kernel(const int32_t* __restrict__ table, const int32_t* __restrict__ q_start,
+                                     int q_per_seq, int B, int max_blocks, int num_blocks, int32_t* __restrict__ rows) {
+  pdl_trigger();
+  pdl_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= B * max_blocks) return;
+  const int b = i / max_blocks, j = i % max_blocks;
+  int r = -1;
+  if (j * 64 < q_start[b] + q_per_seq) {
+    const int blk = table[i];
+    if (blk >= 0 && blk < num_blocks) r = blk * 64;
+    else record_error(ERR_CAPACITY, 704);
+  }
+  rows[i] = r;
+}
+
+// Scratch of the un-absorbed prefill: page rows and the decompressed keys
+// and values of every pool row, [num_blocks * 64][2 * n_h * d_h] bf16.
+inline size_t ws_prefill_unabsorbed(const mla_layer_desc* D, int num_blocks, int B, int max_blocks) {
+  Carver c{nullptr, 0};
+  c.take((size_t)B * max_blocks * 4);
+  c.take((size_t)num_blocks * 64 * 2 * D->n_h * D->d_h * 2);
+  return c.used + 256;
+}
+
+static mla_status_t tc_prefill_unabsorbed(const mla_layer_desc* D, const mla_weights* w, const void* q_c,
+                                          const void* q_rope, const mla_paged_cache* cache, const int32_t* q_start,
+                                          int q_per_seq, int B, void* ws, size_t ws_bytes, void* o, float* lse,
+                                          cudaStream_t st) {
+  if (D->d_h != 128 || !aligned16(q_c) || !aligned16(q_rope) || !aligned16(o) || !aligned16(w->w_uk) ||
+      !aligned16(w->w_uv) || !aligned16(cache->pool))
+    return D->d_h != 128 ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+  Carver cv = carve(ws, ws_bytes);
+  int32_t* rows = (int32_t*)cv.take((size_t)B * cache->max_blocks * 4);
+  __nv_bfloat16* kv = (__nv_bfloat16*)cv.take((size_t)cache->num_blocks * 64 * 2 * D->n_h * D->d_h * 2);
+  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
+  const int n_pages = B * cache->max_blocks;
+  if (launch_pdl(mla_page_rows_kernel, dim3((n_pages + 255) / 256), dim3(256), 0, st, 1, cache->block_table, q_start,
+                 q_per_seq, B, cache->max_blocks, cache->num_blocks, rows) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  const int nq = D->n_h * D->d_h;
+  {  // [k^C ; v^C] of every page of the chunk's sequences: [W^UK ; W^UV] c^KV (eqs 10-11)
+    GemmCall c{};
+    c.a0 = w->w_uk;
+    c.rows0 = nq;
+    c.a1 = w->w_uv;
+    c.rows1 = nq;
+    c.a_row_elems = D->d_c;
+    c.x = cache->pool;
+    c.x_rows = (long long)cache->num_blocks * 64;
+    c.x_row_elems = D->d_c;  // the c^KV columns of each [c^KV | k^R] row
+    c.K = D->d_c;
+    c.T = cache->num_blocks * 64;
+    c.Z = 1;
+    c.b_tile_row = rows;
+    c.n_tiles_override = n_pages;
+    GemmEpi e{};
+    e.kind = EPI_BF16;
+    e.out = kv;
+    e.out_t = 2LL * nq;
+    GemmPlan p;
+    p.tn = 64;  // one cache page per token tile
+    p.n_tiles = n_pages;
+    p.deep = false;
+    p.splits = 1;
+    p.kcs = D->d_c / GEMM_BK;
+    mla_status_t s = run_gemm_paged(c, e, p, (uint64_t)(D->d_c + D->d_hr) * 2, st);
+    if (s != MLA_OK) return s;
+  }
+  CUtensorMap mq, mr, mkv, mkr;
+  const long long T = (long long)B * q_per_seq;
+  bool ok = map_2d(&mq, q_c, (uint64_t)nq, (uint64_t)T, (uint64_t)nq * 2, 64, 128);
+  ok = ok && map_2d(&mr, q_rope, (uint64_t)D->n_h * D->d_hr, (uint64_t)T, (uint64_t)D->n_h * D->d_hr * 2, 64, 128);
+  ok = ok && map_2d(&mkv, kv, 2ULL * nq, (uint64_t)cache->num_blocks * 64, 4ULL * nq, 64, 64);
+  ok = ok && map_2d(&mkr, cache->pool, (uint64_t)(D->d_c + D->d_hr), (uint64_t)cache->num_blocks * 64,
+                    (uint64_t)(D->d_c + D->d_hr) * 2, 64, 64);
+  if (!ok) return MLA_ERR_CUDA;
+  PrefillArgs a;
+  a.n_h = D->n_h;
+  a.q_per_seq = q_per_seq;
+  a.num_blocks = cache->num_blocks;
+  a.max_blocks = cache->max_blocks;
+  a.scale_log2 = (float)(D->attn_logit_factor / sqrt((double)(D->d_h + D->d_hr)) * 1.4426950408889634);
+  a.table = cache->block_table;
+  a.q_start = q_start;
+  a.o = (__nv_bfloat16*)o;
+  a.lse = lse;
+  cudaFuncSetAttribute(mla_prefill_unabsorbed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PfCfg::SMEM);
+  const dim3 grid((q_per_seq + 127) / 128, D->n_h, B);
+  return launch_pdl(mla_prefill_unabsorbed_kernel, grid, dim3(PfCfg::THREADS), PfCfg::SMEM, st, 1, mq, mr, mkv, mkr,
+                    a) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
 }

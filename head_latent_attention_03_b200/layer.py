@@ -18,6 +18,30 @@ import torch
 from . import mla
 
 
+def prefill_flops(dims, prior_lens, q_per_seq: int) -> Dict[str, int]:
+    """FLOPs of the attention of a prefill chunk in each form.
+
+    Latent (absorbed) form: 2 n_h (2 d_c + d_h^R) per (query, key) pair.
+    Un-absorbed form: 2 n_h (2 d_h + d_h^R) per pair, plus the decompression
+    of every cached row of the chunk's sequences into per-head keys and values
+    (2 * 2 n_h d_h d_c per row).
+    """
+    pairs = sum(int(L) * q_per_seq + q_per_seq * (q_per_seq + 1) // 2 for L in prior_lens)
+    rows = sum(int(L) + q_per_seq for L in prior_lens)
+    D = dims
+    return {"absorbed": pairs * 2 * D.n_h * (2 * D.d_c + D.d_hr),
+            "unabsorbed": pairs * 2 * D.n_h * (2 * D.d_h + D.d_hr) + rows * 4 * D.n_h * D.d_h * D.d_c}
+
+
+def cheaper_prefill_form(dims, prior_lens, q_per_seq: int) -> str:
+    """The form with fewer FLOPs for this chunk (bf16 layers with d_h = 128
+    have both; others only the absorbed one)."""
+    if dims.dtype != "bf16" or dims.d_h != 128:
+        return "absorbed"
+    f = prefill_flops(dims, prior_lens, q_per_seq)
+    return "unabsorbed" if f["unabsorbed"] < f["absorbed"] else "absorbed"
+
+
 def torch_dtype(dims) -> torch.dtype:
     return torch.bfloat16 if dims.dtype == "bf16" else torch.float32
 
@@ -110,4 +134,27 @@ class MLALayer:
         self.absorb_q(st, stream)
         self.attend(st, num_splits, stream)
         self.out_proj(st, stream)
+        return st.u
+
+    # un-absorbed chunked prefill ---------------------------------------------
+    def prefill_buffers(self, st: DecodeState):
+        """q^C, per-head o and the decompression workspace of the un-absorbed form."""
+        D, dev = self.dims, self.device
+        T = st.h.shape[0]
+        if not hasattr(st, "q_c"):
+            st.q_c = torch.empty((T, D.n_h, D.d_h), dtype=torch.bfloat16, device=dev)
+            st.o = torch.empty((T, D.n_h, D.d_h), dtype=torch.bfloat16, device=dev)
+            ws = mla.prefill_unabsorbed_workspace_size(self.desc, st.pool.shape[0], st.table.shape[0],
+                                                       st.table.shape[1])
+            st.ws_pf = torch.empty((ws,), dtype=torch.uint8, device=dev)
+        return st
+
+    def prefill_step_unabsorbed(self, st: DecodeState, stream=None) -> torch.Tensor:
+        """Append, queries without absorption, un-absorbed causal attention, W^O."""
+        self.prefill_buffers(st)
+        self.compress_append(st, stream)
+        mla.queries(self.desc, self.cw, st.h, st.pos, st.q_c, st.q_rope, st.ws, stream)
+        mla.prefill_attn_unabsorbed(self.desc, self.cw, st.q_c, st.q_rope, self.cache(st), st.q_start,
+                                    st.new_per_seq, st.ws_pf, st.o, st.lse, stream)
+        mla.out_proj_unabsorbed(self.desc, self.cw, st.o, st.u, stream)
         return st.u

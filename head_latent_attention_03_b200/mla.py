@@ -79,6 +79,18 @@ _SIGS = {
                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                     ctypes.c_void_p]),
     "mla_get_last_error": (ctypes.c_int, [ctypes.c_void_p]),
+    "mla_prefill_unabsorbed_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(LayerDesc), ctypes.c_int,
+                                                                ctypes.c_int, ctypes.c_int]),
+    "mla_queries": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_size_t, ctypes.c_void_p]),
+    "mla_prefill_attn_unabsorbed": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights),
+                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(PagedCache),
+                                                   ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                                   ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p,
+                                                   ctypes.c_void_p]),
+    "mla_out_proj_unabsorbed": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
+                                               ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -202,6 +214,32 @@ def out_proj(desc, w: Weights, o_lat, u, ws, stream=None):
     _check("mla_out_proj", lib().mla_out_proj(
         ctypes.byref(desc), ctypes.byref(w), _ptr(o_lat), o_lat.shape[0], _ptr(u), _ptr(ws),
         ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def prefill_unabsorbed_workspace_size(desc: LayerDesc, num_blocks: int, B: int, max_blocks: int) -> int:
+    return lib().mla_prefill_unabsorbed_workspace_size(ctypes.byref(desc), num_blocks, B, max_blocks)
+
+
+def queries(desc, w: Weights, h, pos, q_c, q_rope, ws, stream=None):
+    """q^C [T, n_h, d_h] and RoPE'd q^R [T, n_h, d_hr] without the W^UK absorption."""
+    _check("mla_queries", lib().mla_queries(
+        ctypes.byref(desc), ctypes.byref(w), _ptr(h), _ptr(pos), h.shape[0], _ptr(q_c), _ptr(q_rope), _ptr(ws),
+        ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def prefill_attn_unabsorbed(desc, w: Weights, q_c, q_rope, cache: PagedCache, q_start, q_per_seq, ws, o, lse=None,
+                            stream=None):
+    """Causal attention of a prefill chunk with decompressed per-head keys and values: o [T, n_h, d_h]."""
+    _check("mla_prefill_attn_unabsorbed", lib().mla_prefill_attn_unabsorbed(
+        ctypes.byref(desc), ctypes.byref(w), _ptr(q_c), _ptr(q_rope), ctypes.byref(cache), _ptr(q_start), q_per_seq,
+        q_start.shape[0], _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _ptr(o), _ptr(lse),
+        _stream(stream)))
+
+
+def out_proj_unabsorbed(desc, w: Weights, o, u, stream=None):
+    """u = W^O o for per-head outputs o [T, n_h, d_h]."""
+    _check("mla_out_proj_unabsorbed", lib().mla_out_proj_unabsorbed(
+        ctypes.byref(desc), ctypes.byref(w), _ptr(o), o.shape[0], _ptr(u), _stream(stream)))
 
 
 def get_last_error(stream=None) -> int:

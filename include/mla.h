@@ -229,6 +229,34 @@ mla_status_t mla_prefill_attn(const mla_layer_desc* desc, const void* q_lat, con
                               const mla_paged_cache* cache, const int32_t* q_start, int q_per_seq, int B,
                               void* ws, size_t ws_bytes, void* o_lat, float* lse, void* stream);
 
+/* Chunked prefill in the un-absorbed form (the reading notes' eqs 10-11: per-head
+ * keys k^C_i = W^UK_i c^KV and values v^C_i = W^UV_i c^KV decompressed once per
+ * chunk, then causal attention with q_i = [q^C_i ; q^R_i], k_i = [k^C_i ; k^R]).
+ * Per (query, key) pair it costs 2 n_h (d_h + d_h^R + d_h) FLOP against
+ * 2 n_h (2 d_c + d_h^R) in the latent form, plus the decompression of every
+ * cached row of the chunk's sequences: cheaper for long chunks.
+ *
+ * mla_queries: q_c [T, n_h, d_h] and q_rope [T, n_h, d_hr] (eqs 12-13, decoupled
+ *   query), without the W^UK absorption.  Workspace as mla_absorb_q's.
+ * mla_prefill_attn_unabsorbed: after mla_compress_append of the chunk, query q
+ *   of sequence b at position q_start[b] + q attends rows 0 .. q_start[b] + q.
+ *   Decompresses the pages of rows 0 .. q_start[b] + q_per_seq - 1 of each
+ *   sequence into the workspace (mla_prefill_unabsorbed_workspace_size bytes:
+ *   2 n_h d_h bf16 values per pool row), then runs the attention.
+ *   q_c, q_rope [B*q_per_seq, n_h, ...] from mla_queries; o [B*q_per_seq, n_h,
+ *   d_h] bf16 out; lse [B*q_per_seq, n_h] float out (may be NULL).  bf16 layers
+ *   with d_h == 128.
+ * mla_out_proj_unabsorbed: u [T, d] float = W^O o (eq 8) for o [T, n_h, d_h]. */
+size_t mla_prefill_unabsorbed_workspace_size(const mla_layer_desc* desc, int num_blocks, int B, int max_blocks);
+mla_status_t mla_queries(const mla_layer_desc* desc, const mla_weights* w, const void* h, const int32_t* pos, int T,
+                         void* q_c, void* q_rope, void* ws, size_t ws_bytes, void* stream);
+mla_status_t mla_prefill_attn_unabsorbed(const mla_layer_desc* desc, const mla_weights* w, const void* q_c,
+                                         const void* q_rope, const mla_paged_cache* cache, const int32_t* q_start,
+                                         int q_per_seq, int B, void* ws, size_t ws_bytes, void* o, float* lse,
+                                         void* stream);
+mla_status_t mla_out_proj_unabsorbed(const mla_layer_desc* desc, const mla_weights* w, const void* o, int T, float* u,
+                                     void* stream);
+
 /* Output projection (eq 8 with W^UV absorbed): u = W^O [W^UV_i o_lat_i]_i.
  *   o_lat [T, n_h, d_c]; u [T, d] float                                     */
 mla_status_t mla_out_proj(const mla_layer_desc* desc, const mla_weights* w, const void* o_lat, int T,

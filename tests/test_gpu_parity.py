@@ -339,3 +339,51 @@ def test_context_parallel_long_context():
     _, _, _, o, l = _cp_merge(layer, st, batch, 4)
     assert_bf16(np32(o), np32(st.o_lat), "merged vs one-GPU decode")
     assert np.max(np.abs(np32(l) - np32(st.lse))) < 2e-2
+
+
+# ----------------------------------------------------------------------------
+# un-absorbed chunked prefill: decompressed per-head keys and values, causal
+# flash attention, W^O; against the oracle's un-absorbed form (eqs 10-11)
+# ----------------------------------------------------------------------------
+def _unabsorbed(w, batch):
+    layer = MLALayer(w.dims, weights_for(w))
+    st = layer.upload(batch)
+    layer.prefill_step_unabsorbed(st)
+    torch.cuda.synchronize()
+    code = mla.get_last_error()
+    assert code == 0, mla.status_string(code)
+    return layer, st
+
+
+def _check_unabsorbed(w, batch, st, seqs_queries):
+    D, W = w.dims, weights_for(w)
+    n = w.new_tokens
+    for b, qs in seqs_queries:
+        L = int(batch.prior_len[b])
+        prior = O.gather_rows(batch.pool, batch.block_table[b], L, D.block_size)
+        new_r, outs = O.prefill_sequence(D, W, batch.h[b * n:(b + 1) * n], L, prior, qs, absorbed=False)
+        assert_bf16(new_rows(st, batch)[b * n:(b + 1) * n], new_r, "rows")
+        for q in qs:
+            r = b * n + q
+            assert_bf16(np32(st.o)[r], outs[q]["o"], f"o b={b} q={q}")
+            assert np.max(np.abs(np32(st.lse)[r] - outs[q]["lse"])) < 2e-2
+            assert_bf16(np32(st.u)[r], outs[q]["u"], f"u b={b} q={q}")
+
+
+def test_unabsorbed_prefill_small():
+    # 200 new queries (two query blocks, the second partial) over 100 and 300
+    # prior rows; the last page of each sequence is partly unwritten (NaN)
+    w = dataclasses.replace(I.WORKLOADS["prefill"], name="pf_small", batch=2, prior="list:100,300", new_tokens=200)
+    batch = I.gen_batch(w)
+    layer, st = _unabsorbed(w, batch)
+    _check_unabsorbed(w, batch, st, [(0, list(range(0, 200, 7)) + [199]), (1, [0, 27, 63, 64, 127, 128, 199])])
+    # the latent form of the same chunk gives the same layer output
+    _, st2 = run_gpu(w, batch)
+    assert_bf16(np32(st.u), np32(st2.u), "un-absorbed vs absorbed u")
+
+
+def test_unabsorbed_prefill_full_size_sampled():
+    w = I.WORKLOADS["prefill"]
+    batch = I.gen_batch(w)
+    layer, st = _unabsorbed(w, batch)
+    _check_unabsorbed(w, batch, st, [(5, [0, 1, 127, 128, 2047, 4095]), (0, [63, 64, 4094])])
