@@ -236,35 +236,69 @@ def workload_work(w, batch):
     return bytes_, flops
 
 
+def unabsorbed_work(w, batch):
+    """Algorithmic bytes and FLOPs of the un-absorbed prefill attention: the
+    per-head products 2 n_h (2 d_h + d_h^R) per (query, key) pair plus the
+    decompression of every cached row (2 x 2 n_h d_h d_c); bytes = the cached
+    rows, q^C, q^R and o once."""
+    from head_latent_attention_03_b200.layer import prefill_flops
+    D = w.dims
+    flops = prefill_flops(D, batch.prior_len, w.new_tokens)["unabsorbed"]
+    rows = batch.h.shape[0]
+    cached = int(sum(int(L) + w.new_tokens for L in batch.prior_len))
+    bytes_ = cached * D.row * 2 + rows * D.n_h * (2 * D.d_h + D.d_hr) * 2
+    return bytes_, flops
+
+
 def measure_extra(name, steps, warmup, dev, peaks, peak_src):
     """One more workload of the scope in the same run: whole-step and
-    attention-stage device times (CUDA events, max over ranks)."""
+    attention-stage device times (CUDA events, max over ranks).  A prefill
+    chunk runs in the form with fewer FLOPs (layer.cheaper_prefill_form)."""
     import torch
     from head_latent_attention_03_b200 import inputs as I, mla
-    from head_latent_attention_03_b200.layer import MLALayer
+    from head_latent_attention_03_b200.layer import MLALayer, cheaper_prefill_form
     w = I.WORKLOADS[name]
     batch = I.gen_batch(w)
     layer = MLALayer(w.dims, I.gen_weights(w), device=str(dev))
     st = layer.upload(batch)
     rows = st.h.shape[0]
-    attn_bytes, attn_flops = workload_work(w, batch)
+    form = cheaper_prefill_form(w.dims, batch.prior_len, w.new_tokens) if w.new_tokens > 1 else "absorbed"
+    if form == "unabsorbed":
+        attn_bytes, attn_flops = unabsorbed_work(w, batch)
+        layer.prefill_buffers(st)
+        calls = [lambda: layer.compress_append(st),
+                 lambda: mla.queries(layer.desc, layer.cw, st.h, st.pos, st.q_c, st.q_rope, st.ws)]
+        attend = lambda: mla.prefill_attn_unabsorbed(layer.desc, layer.cw, st.q_c, st.q_rope, layer.cache(st),
+                                                     st.q_start, st.new_per_seq, st.ws_pf, st.o, st.lse)
+        after = lambda: mla.out_proj_unabsorbed(layer.desc, layer.cw, st.o, st.u)
+    else:
+        attn_bytes, attn_flops = workload_work(w, batch)
+        calls = [lambda: layer.compress_append(st), lambda: layer.absorb_q(st)]
+        attend = lambda: layer.attend(st)
+        after = lambda: layer.out_proj(st)
     stream = torch.cuda.current_stream()
+
+    def one(k=None):
+        for f in calls:
+            f()
+        if k is not None:
+            ev[k][0].record(stream)
+        attend()
+        if k is not None:
+            ev[k][1].record(stream)
+        after()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for _ in range(warmup):
-        layer.step(st)
+        one()
     torch.cuda.synchronize()
     code = mla.get_last_error()
     if code != 0:
         raise RuntimeError(f"{name}: device status after warm-up: {mla.status_string(code)}")
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for k in range(steps):
-        layer.compress_append(st)
-        layer.absorb_q(st)
-        ev[k][0].record(stream)
-        layer.attend(st)
-        ev[k][1].record(stream)
-        layer.out_proj(st)
+        one(k)
     e1.record(stream)
     torch.cuda.synchronize()
     code = mla.get_last_error()
@@ -277,7 +311,22 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
     out = {"workload": WORKLOAD_TEXT[name], "value": round(world * rows * steps / (t_ms * 1e-3), 1),
            "unit": "tokens/s", "steps": steps, "warmup": warmup, "ms_per_step": round(t_ms / steps, 4),
            "roofline": roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src)}
-    out["roofline"]["traffic"] = committed_traffic(name)
+    out["roofline"]["traffic"] = committed_traffic(name) if form == "absorbed" else None
+    if w.new_tokens > 1:
+        out["form"] = form
+        if form == "unabsorbed":
+            # the latent form of the same chunk, for comparison (attention only)
+            lat_bytes, lat_flops = workload_work(w, batch)
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            layer.absorb_q(st)
+            a0.record(stream)
+            layer.attend(st)
+            a1.record(stream)
+            torch.cuda.synchronize()
+            (lat_ms,) = max_over_ranks([a0.elapsed_time(a1)], dev)
+            out["latent_form_attention"] = {"attn_ms": round(lat_ms, 3),
+                                            "roofline": roofline_of(lat_bytes, lat_flops, lat_ms, peaks, peak_src)}
     del layer, st
     torch.cuda.empty_cache()
     return out
