@@ -48,6 +48,9 @@ class LayerDims:
     norm_eps: float = 1e-6
     scale_kv: float = 1.0
     scale_q: float = 1.0
+    # latent cache storage: "bf16" (the layer's precision) or "fp8" (E4M3
+    # codes of c^KV with one power-of-two scale per row; k^R stays bf16)
+    cache_dtype: str = "bf16"
 
     @property
     def row(self) -> int:
@@ -89,6 +92,8 @@ WORKLOADS: Dict[str, Workload] = {
     "v2": Workload("v2", 3, V2, 64, "uniform:1:8192", permute_pages=True),
     "long": Workload("long", 4, V2_YARN, 4, "fixed:131072"),
     "prefill": Workload("prefill", 5, V2, 8, "fixed:4096", new_tokens=4096),
+    # the V2-Lite workload (same draws) over an FP8 latent cache
+    "lite_fp8": Workload("lite_fp8", 2, dataclasses.replace(LITE, cache_dtype="fp8"), 32, "fixed:4096"),
 }
 
 # tensor ids inside a workload's seed tree

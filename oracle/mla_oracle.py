@@ -38,6 +38,15 @@ explicit choice here, shared by the CUDA path only as a convention):
     gains g and scalar factors s_kv, s_q.  The factor follows the norm (a
     factor in front of it would cancel).  k^R is not a compressed latent and
     is not normalised.
+  * The quantised latent cache ([explainer] 3.1.4 serves V2 with the KV
+    cache quantised to about 6 bits per element; no format is printed), when
+    a layer uses it: each cached c^KV row is stored as FP8 E4M3 codes (OCP
+    8-bit float: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+    subnormals, no infinities, largest finite 448) times one power-of-two
+    scale 2^e per row, e the smallest integer with max|c| <= 448 * 2^e, codes
+    rounded to nearest with ties to even and saturated at +-448.  k^R stays
+    in the layer's precision (positions need its bits).  The attention reads
+    the dequantised row codes * 2^e.
 
 Every function is fp64 and written for clarity, not speed.
 """
@@ -120,6 +129,71 @@ def latent_norm(D, W, c: np.ndarray, which: str) -> np.ndarray:
     gain = W["g_kv"] if which == "kv" else W["g_q"]
     scale = D.scale_kv if which == "kv" else D.scale_q
     return scale * rms_norm(c, gain, D.norm_eps)
+
+
+# ---------------------------------------------------------------------------
+# quantised latent cache, [explainer] 3.1.4 (KV cache quantisation for serving)
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0    # largest finite E4M3 value, 1.75 * 2^8
+E4M3_MIN_EXP = -6   # exponent of the smallest normal E4M3 value (1 - bias)
+E4M3_MANT = 3       # stored mantissa bits
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """Nearest FP8 E4M3 value of each element, ties to even, saturated to +-448.
+
+    In the binade [2^k, 2^(k+1)) the representable values are 2^(k-3) apart;
+    below 2^-6 (subnormals) they are 2^-9 apart.  Rounding the quotient by
+    that spacing to the nearest integer, halves to even, rounds the stored
+    mantissa to nearest even; a quotient that reaches 16 is the next binade's
+    first value.
+    """
+    x = np.asarray(x, dtype=F64)
+    a = np.abs(x)
+    _, k = np.frexp(a)                          # a = f 2^k with f in [0.5, 1)
+    exp = np.maximum(k - 1, E4M3_MIN_EXP)
+    step = np.ldexp(1.0, exp - E4M3_MANT)
+    q = np.round(a / step) * step               # numpy rounds halves to even
+    q = np.minimum(q, E4M3_MAX)
+    return np.copysign(q, x)
+
+
+def fp8_scale_exponent(amax: float) -> int:
+    """Smallest integer e with amax <= 448 * 2^e (0 for a zero row): the row's
+    largest magnitude lands in the top binade of E4M3."""
+    if not amax > 0.0:
+        return 0
+    _, k = math.frexp(amax)                     # amax in [2^(k-1), 2^k)
+    e = (k - 1) - 8                             # 448 * 2^e = 1.75 * 2^(k-1)
+    if amax > E4M3_MAX * 2.0 ** e:
+        e += 1
+    return e
+
+
+def quantize_latent(c: np.ndarray) -> Tuple[np.ndarray, int]:
+    """One cached c^KV row as (E4M3 code values, e), c ~ codes * 2^e."""
+    c = np.asarray(c, dtype=F64)
+    e = fp8_scale_exponent(float(np.max(np.abs(c))))
+    return e4m3_round(np.ldexp(c, -e)), e
+
+
+def cached_row(D, row: np.ndarray) -> np.ndarray:
+    """A cache row [c^KV ; k^R] as the attention reads it back: with the FP8
+    cache c^KV is dequantised from its codes, k^R is kept."""
+    row = np.asarray(row, dtype=F64)
+    if getattr(D, "cache_dtype", "bf16") != "fp8":
+        return row
+    codes, e = quantize_latent(row[:D.d_c])
+    return np.concatenate([np.ldexp(codes, e), row[D.d_c:]])
+
+
+def cached_rows(D, rows: np.ndarray) -> np.ndarray:
+    """cached_row of every row of rows [L, d_c + d_hr]."""
+    rows = np.asarray(rows, dtype=F64)
+    if getattr(D, "cache_dtype", "bf16") != "fp8":
+        return rows
+    return np.stack([cached_row(D, r) for r in rows]) if len(rows) else rows
 
 
 def compress_kv(D, W: Dict[str, np.ndarray], h_t: np.ndarray, pos: int) -> np.ndarray:
@@ -284,13 +358,14 @@ def gather_rows(pool: np.ndarray, table_row: np.ndarray, n: int, block: int) -> 
 def decode_token(D, W, h_t: np.ndarray, pos: int, prior_rows: np.ndarray, absorbed: bool = False) -> Dict[str, np.ndarray]:
     """One new token at position `pos` attending over prior rows + itself.
 
-    Returns the new cache row, q^C, q^R, (absorbed only) q_lat and o_lat,
-    lse and u.
+    Returns the new cache row (and as the attention reads it back from the
+    cache: "row_cached"), q^C, q^R, (absorbed only) q_lat and o_lat, lse and
+    u.  With the FP8 cache every row, prior and new, is read back dequantised.
     """
     row = compress_kv(D, W, h_t, pos)
-    rows = np.concatenate([np.asarray(prior_rows, dtype=F64), row[None, :]], axis=0)
+    rows = cached_rows(D, np.concatenate([np.asarray(prior_rows, dtype=F64), row[None, :]], axis=0))
     q_c, q_r = queries(D, W, h_t, pos)
-    out = {"row": row, "q_c": q_c, "q_r": q_r}
+    out = {"row": row, "row_cached": rows[-1], "q_c": q_c, "q_r": q_r}
     if absorbed:
         q_lat = absorb_query(D, W, q_c)
         o_lat, lse, u = attend_absorbed(D, W, q_lat, q_r, rows)
@@ -322,7 +397,7 @@ def prefill_sequence(D, W, h_new: np.ndarray, start: int, prior_rows: np.ndarray
     (q_lat, o_lat, lse, u) (absorbed) or (o, lse, u).
     """
     new_rows = np.stack([compress_kv(D, W, h_new[q], start + q) for q in range(len(h_new))])
-    rows = np.concatenate([np.asarray(prior_rows, dtype=F64), new_rows], axis=0)
+    rows = cached_rows(D, np.concatenate([np.asarray(prior_rows, dtype=F64), new_rows], axis=0))
     outs = {}
     for q in query_ids:
         pos = start + q

@@ -462,3 +462,99 @@ def test_merged_partials_equal_attention_over_all_rows():
     o, lse = O.merge_partials(parts_o, parts_l)
     assert np.max(np.abs(o - full_o)) <= 1e-12 * np.max(np.abs(full_o))
     assert np.max(np.abs(lse - full_lse)) <= 1e-12 * np.max(np.abs(full_lse))
+
+
+# 13. the quantised latent cache ([explainer] 3.1.4: the KV cache is
+# quantised for serving).  The format (FP8 E4M3 codes of c^KV, one
+# power-of-two scale per row, k^R kept) is a reading; the pins below fix the
+# arithmetic of that reading from the format's bit-level definition, not from
+# the oracle's own formula.
+
+def _e4m3_table():
+    """Every finite E4M3 value from its bit fields (sign, 4-bit exponent with
+    bias 7, 3-bit mantissa; exponent field 0 = subnormal; S.1111.111 = NaN),
+    with the mantissa field of each."""
+    vals, mants = [], []
+    for bits in range(256):
+        s, E, m = bits >> 7, (bits >> 3) & 15, bits & 7
+        if E == 15 and m == 7:
+            continue
+        v = (m / 8.0) * 2.0 ** -6 if E == 0 else (1.0 + m / 8.0) * 2.0 ** (E - 7)
+        vals.append(-v if s else v)
+        mants.append(m)
+    return np.array(vals), np.array(mants)
+
+
+def _e4m3_brute(x):
+    """Nearest finite E4M3 value by search; a tie goes to the even mantissa
+    field; magnitudes past the largest value saturate to it."""
+    vals, mants = _e4m3_table()
+    out = np.empty_like(x)
+    top = np.max(vals)
+    for i, v in enumerate(x):
+        if abs(v) >= top:
+            out[i] = math.copysign(top, v)
+            continue
+        d = np.abs(vals - v)
+        best = np.flatnonzero(d == d.min())
+        if len(best) > 1:
+            best = [b for b in best if mants[b] % 2 == 0 and (vals[b] != 0 or math.copysign(1, vals[b]) == math.copysign(1, v))] or best
+        out[i] = vals[best[0]]
+    return out
+
+
+def test_e4m3_rounding_matches_search_over_all_codes():
+    vals, _ = _e4m3_table()
+    assert np.max(vals) == 448.0 and len(np.unique(vals)) == 253  # 254 finite codes, +0 and -0 equal
+    pos = np.unique(vals[vals > 0])
+    mids = (pos[:-1] + pos[1:]) / 2  # every tie between neighbours
+    rng = np.random.default_rng(13)
+    mags = np.ldexp(rng.uniform(1.0, 2.0, 3000), rng.integers(-12, 10, 3000))
+    x = np.concatenate([mids, -mids, pos, mags, -mags, [0.0, 2.0 ** -10, 460.0, 464.0, 500.0, 1e4]])
+    got = O.e4m3_round(x)
+    want = _e4m3_brute(x)
+    assert np.array_equal(got, want), x[got != want][:5]
+
+
+def test_e4m3_worked_values():
+    # hand-computed: 1.0625 lies halfway between 1 (mantissa 000) and 1.125
+    # (001) -> 1; 1.1875 between 1.125 (001) and 1.25 (010) -> 1.25; 3 * 2^-10
+    # between the subnormals 2^-9 (001) and 2^-8 (010) -> 2^-8; 2^-10 between
+    # 0 and 2^-9 -> 0; 464 between 448 and the missing 480 -> 448 (saturated)
+    x = np.array([1.0625, 1.1875, 3 * 2.0 ** -10, 2.0 ** -10, 464.0, 1000.0, -1.0625, 240.0, 0.3, 2.0 ** -9])
+    want = np.array([1.0, 1.25, 2.0 ** -8, 0.0, 448.0, 448.0, -1.0, 240.0, 0.3125, 2.0 ** -9])
+    assert np.array_equal(O.e4m3_round(x), want)
+
+
+def test_fp8_row_scale_uses_the_top_binade():
+    rng = np.random.default_rng(14)
+    for _ in range(200):
+        c = rng.standard_normal(512) * 2.0 ** rng.uniform(-20, 20)
+        amax = np.max(np.abs(c))
+        codes, e = O.quantize_latent(c)
+        assert 224.0 < amax * 2.0 ** -e <= 448.0
+        # largest code in the top binade, nothing saturated beyond rounding
+        assert 224.0 <= np.max(np.abs(codes)) <= 448.0
+        back = codes * 2.0 ** e
+        normal = np.abs(c) * 2.0 ** -e >= 2.0 ** -6
+        # normal values: half a spacing of 2^-3 relative; subnormals: 2^-10 * 2^e
+        assert np.all(np.abs(back - c)[normal] <= 2.0 ** -4 * np.abs(c)[normal])
+        assert np.all(np.abs(back - c)[~normal] <= 2.0 ** (e - 10))
+    assert O.fp8_scale_exponent(448.0) == 0 and O.fp8_scale_exponent(448.5) == 1
+    assert O.fp8_scale_exponent(1.75) == -8 and O.fp8_scale_exponent(0.0) == 0
+
+
+def test_fp8_cached_row_keeps_k_rope_and_is_a_fixed_point():
+    import dataclasses
+    D = dataclasses.replace(LITE, cache_dtype="fp8")
+    rng = np.random.default_rng(15)
+    row = rng.standard_normal(D.row)
+    once = O.cached_row(D, row)
+    assert np.array_equal(once[D.d_c:], row[D.d_c:])
+    assert not np.array_equal(once[:D.d_c], row[:D.d_c])
+    # read back at the row's own magnitude: within half an E4M3 spacing
+    # (2^-4 relative) of the largest element
+    assert np.max(np.abs(once[:D.d_c] - row[:D.d_c])) <= 2.0 ** -4 * np.max(np.abs(row[:D.d_c]))
+    assert np.array_equal(O.cached_row(D, once), once)
+    # the bf16 cache reads rows back unchanged
+    assert np.array_equal(O.cached_row(LITE, row), row)

@@ -57,6 +57,20 @@ MUTATIONS = {
     "merge_unnormalised": ("/ tot[..., None]", ""),
     # merge weighing the parts equally
     "merge_equal_weights": ("w = np.exp(lse - m)", "w = np.ones_like(lse)"),
+    # FP8 cache: halves rounded away from zero instead of to even
+    "e4m3_ties_away": ("q = np.round(a / step) * step", "q = np.floor(a / step + 0.5) * step"),
+    # FP8 cache: no subnormal range (the spacing keeps shrinking below 2^-6)
+    "e4m3_no_subnormals": ("exp = np.maximum(k - 1, E4M3_MIN_EXP)", "exp = k - 1"),
+    # FP8 cache: the largest value of a format with exponent bias 8
+    "e4m3_wrong_bias": ("E4M3_MAX = 448.0 ", "E4M3_MAX = 240.0 "),
+    # FP8 cache: scale exponent rounded down (the row maximum saturates)
+    "fp8_scale_rounded_down": ("    if amax > E4M3_MAX * 2.0 ** e:\n        e += 1\n", ""),
+    # FP8 cache: k^R quantised with the latent
+    "fp8_quantises_rope": ("codes, e = quantize_latent(row[:D.d_c])\n    return np.concatenate([np.ldexp(codes, e), row[D.d_c:]])",
+                           "codes, e = quantize_latent(row)\n    return np.ldexp(codes, e)"),
+    # FP8 cache: codes read back without their scale
+    "fp8_scale_not_applied": ("return np.concatenate([np.ldexp(codes, e), row[D.d_c:]])",
+                              "return np.concatenate([codes, row[D.d_c:]])"),
     # W^O applied before W^UV's head split is undone
     "out_proj_heads": ("o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64))",
                        "o = np.einsum(\"ihc,ic->ih\", w_uv, np.asarray(o_lat, dtype=F64)[::-1])"),
