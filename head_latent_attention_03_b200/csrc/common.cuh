@@ -464,6 +464,53 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------------------
+// FP8 latent cache rows (KV cache quantisation for serving, DeepSeek-V2
+// explainer, adg.csdn.net, section 3.1.4; the format is this library's):
+//   [E4M3 codes of c^KV (d_c bytes) | k^R (d_hr bf16) | fp32 scale 2^e | pad]
+// the row padded to a multiple of 16 bytes (656 bytes at d_c 512, d_hr 64).
+// E4M3 = OCP 8-bit float, 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+// bits, largest finite 448.  e is the smallest integer with
+// max|c| <= 448 * 2^e, so the row maximum lands in the top binade.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int fp8_row_bytes(int d_c, int d_hr) { return (d_c + 2 * d_hr + 4 + 15) / 16 * 16; }
+__host__ __device__ constexpr int fp8_scale_off(int d_c, int d_hr) { return d_c + 2 * d_hr; }
+
+// 2^e as a float, e in [-126, 127]
+__device__ __forceinline__ float exp2_int(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// Scale exponent of a row whose largest magnitude is amax (0 for a zero row),
+// kept in [-126, 126] so that 2^e and 2^-e are normal floats.
+__device__ __forceinline__ int fp8_scale_exponent(float amax) {
+  if (!(amax > 0.f)) return 0;
+  const int biased = (int)((__float_as_uint(amax) >> 23) & 0xFFu);
+  int e = (biased == 0 ? -127 : biased - 127) - 8;  // floor(log2 amax) - 8: 448 * 2^e = 1.75 * 2^floor
+  if (e < -126) e = -126;
+  if (e <= 119 && amax > 448.f * exp2_int(e)) ++e;
+  return e > 126 ? 126 : e;
+}
+
+// Two floats to two E4M3 codes, round to nearest even, saturated to +-448;
+// lo lands in the low byte.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 codes (low byte = element 0) times 2^e as two bf16 (element 0 in
+// the low half), exactly: the codes become f16 (every E4M3 value is a normal
+// f16 except 0), and the f16 exponent field is rebased to bf16's bias plus e
+// (bias_e = (112 + e) << 7; the f16 mantissa's three used bits shift into
+// bf16's top mantissa bits).  Zeros stay zero.  Exact for e >= -112.
+__device__ __forceinline__ uint32_t bf16x2_from_e4m3x2(uint16_t codes, uint32_t bias_e) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(codes));
+  const uint32_t mag = h & 0x7FFF7FFFu;
+  const uint32_t nz = ((mag + 0x7FFF7FFFu) >> 15) & 0x00010001u;  // 1 in each non-zero half
+  return ((mag >> 3) + nz * bias_e) | (h & 0x80008000u);
+}
+
 // Byte offset inside a swizzled (SW32/64/128) region: the 16-byte chunk index
 // (bits 4..6) is XORed with the 128-byte row index (bits 7..9), masked to the
 // swizzle width.

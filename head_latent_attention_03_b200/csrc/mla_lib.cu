@@ -35,8 +35,14 @@ bool desc_valid(const mla_layer_desc* D) {
   if (!(D->rope_base > 0.0) || !(D->yarn_scale >= 1.0) || !(D->attn_logit_factor > 0.0)) return false;
   if (D->yarn_scale > 1.0 && (D->yarn_orig_ctx <= 0 || !(D->yarn_beta > D->yarn_alpha))) return false;
   if (D->latent_norm && (!(D->norm_eps >= 0.0) || !(D->scale_kv > 0.0) || !(D->scale_q > 0.0))) return false;
+  if (D->cache_dtype != MLA_CACHE_NATIVE && !(D->cache_dtype == MLA_CACHE_FP8_E4M3 && D->dtype == MLA_BF16))
+    return false;
   return D->dtype == MLA_F32 || D->dtype == MLA_BF16;
 }
+
+// The latent attention kernels that read FP8 rows: the one-CTA kernel
+// (n_h <= 64); the CTA-pair kernel (n_h = 128) reads bf16 rows only.
+bool attn_cache_supported(const mla_layer_desc* D) { return !fp8_cache(D) || !use_pair_kernel(D); }
 
 // Shapes the tcgen05 kernels are written for.
 bool bf16_supported(const mla_layer_desc* D) {
@@ -131,6 +137,29 @@ const char* mla_status_string(mla_status_t s) {
   return "unknown status";
 }
 
+size_t mla_cache_row_bytes(const mla_layer_desc* D) {
+  if (!desc_valid(D)) return 0;
+  if (D->dtype == MLA_F32) return (size_t)(D->d_c + D->d_hr) * sizeof(float);
+  return (size_t)cache_row_bytes(D);
+}
+
+mla_status_t mla_cache_quantize(const mla_layer_desc* D, const void* src, long long n, void* dst, void* stream) {
+  if (!desc_valid(D) || !src || !dst || n < 0 || !fp8_cache(D)) return MLA_ERR_INVALID_ARG;
+  if (n == 0) return MLA_OK;
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  if (!aligned16(src) || !aligned16(dst)) return MLA_ERR_INVALID_ARG;
+  const char* s0 = (const char*)src;
+  const char* d0 = (const char*)dst;
+  if (s0 < d0 + n * cache_row_bytes(D) && d0 < s0 + n * (D->d_c + D->d_hr) * 2) return MLA_ERR_INVALID_ARG;
+  const long long blocks = (n + CVT_ROWS_PER_BLOCK - 1) / CVT_ROWS_PER_BLOCK;
+  if (blocks > 0x7FFFFFFFLL) return MLA_ERR_UNSUPPORTED;
+  return launch_pdl(mla_cache_to_fp8_kernel, dim3((unsigned)blocks), dim3(32 * CVT_ROWS_PER_BLOCK), 0,
+                    as_stream(stream), 1, (const __nv_bfloat16*)src, n, (uint8_t*)dst, cache_row_bytes(D)) ==
+                 cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
 size_t mla_workspace_size(const mla_layer_desc* D, int T, int B, int max_kv_len) {
   if (!desc_valid(D) || T < 0 || B < 0 || max_kv_len < 0) return 0;
   if (D->dtype == MLA_F32) {
@@ -211,7 +240,7 @@ mla_status_t mla_decode_attn(const mla_layer_desc* D, const void* q_lat, const v
   if (D->dtype == MLA_F32)
     return f32_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, ws, ws_bytes, o_lat, lse,
                          as_stream(stream));
-  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  if (!bf16_supported(D) || !attn_cache_supported(D)) return MLA_ERR_UNSUPPORTED;
   return tc_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, ws, ws_bytes, num_splits, o_lat, lse,
                       as_stream(stream));
 }
@@ -232,7 +261,7 @@ mla_status_t mla_decode_attn_noalloc(const mla_layer_desc* D, const void* q_lat,
     return f32_attention(D, q_lat, q_rope, cache, kv_len, nullptr, 1, B, scratch, kNoAllocScratchBytes, o_lat, lse,
                          as_stream(stream));
   }
-  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  if (!bf16_supported(D) || !attn_cache_supported(D)) return MLA_ERR_UNSUPPORTED;
   // The plan's unit list and partials must fit the array: an explicit split
   // count that does not fit is refused; the automatic plan deals the tiles
   // out to the largest number of CTAs (CTA pairs) whose plan fits.
@@ -257,7 +286,7 @@ mla_status_t mla_decode_attn_partial(const mla_layer_desc* D, const void* q_lat,
       !lse_part)
     return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
-  if (D->dtype != MLA_BF16 || !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  if (D->dtype != MLA_BF16 || !bf16_supported(D) || !attn_cache_supported(D)) return MLA_ERR_UNSUPPORTED;
   return tc_attention(D, q_lat, q_rope, cache, kv_end, nullptr, 1, B, ws, ws_bytes, 0, nullptr, lse_part,
                       as_stream(stream), 0, kv_begin, o_part);
 }
@@ -294,7 +323,7 @@ mla_status_t mla_prefill_attn_unabsorbed(const mla_layer_desc* D, const mla_weig
     return MLA_ERR_INVALID_ARG;
   if (B == 0) return MLA_OK;
   if ((long long)B * q_per_seq > (1 << 30)) return MLA_ERR_UNSUPPORTED;
-  if (D->dtype != MLA_BF16 || !bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  if (D->dtype != MLA_BF16 || !bf16_supported(D) || fp8_cache(D)) return MLA_ERR_UNSUPPORTED;
   return tc_prefill_unabsorbed(D, w, q_c, q_rope, cache, q_start, q_per_seq, B, ws, ws_bytes, o, lse,
                                as_stream(stream));
 }
@@ -318,7 +347,7 @@ mla_status_t mla_prefill_attn(const mla_layer_desc* D, const void* q_lat, const 
   if (D->dtype == MLA_F32)
     return f32_attention(D, q_lat, q_rope, cache, nullptr, q_start, q_per_seq, (int)rows, ws, ws_bytes, o_lat, lse,
                          as_stream(stream));
-  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  if (!bf16_supported(D) || !attn_cache_supported(D)) return MLA_ERR_UNSUPPORTED;
   return tc_attention(D, q_lat, q_rope, cache, nullptr, q_start, q_per_seq, (int)rows, ws, ws_bytes, 1, o_lat, lse,
                       as_stream(stream));
 }

@@ -44,8 +44,11 @@ constexpr int ATT_TILE = 128;        // cached tokens per tile (MMA M)
 constexpr int ATT_DC = 512, ATT_DR = 64;
 constexpr float ATT_RESCALE_LOG2 = 8.0f;
 
-template <int H>
+// F8: the cache rows are FP8 (E4M3 codes of c^KV, bf16 k^R, a power-of-two
+// scale per row); four more warps turn the codes into the bf16 tile.
+template <int H, bool F8 = false>
 struct AttnCfg {
+  static constexpr int THREADS = F8 ? ATT_THREADS + 128 : ATT_THREADS;
   static constexpr int Q_CHUNK = H * 128;              // one 64-column chunk of H rows
   static constexpr int Q_BYTES = 9 * Q_CHUNK;
   static constexpr int P_BYTES = ATT_TILE * 2 * H;     // P^T[128 tokens x H] bf16
@@ -57,13 +60,18 @@ struct AttnCfg {
   static constexpr int OFF_P = OFF_Q + Q_BYTES;
   static constexpr int OFF_ROPE = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_LAT = OFF_ROPE + NR * ROPE_SLOT;
-  static constexpr int OFF_BAR = OFF_LAT + NL * LAT_SLOT;
-  static constexpr int N_BAR = 2 * NL + 2 * NR + 1 + 2 + 2 + 2 + 2 + 1;
+  static constexpr int SC_SLOT = 2048;                 // F8: 2 pages x 64 rows x 16 bytes (scale + padding)
+  static constexpr int NSC = F8 ? 2 : 0;               // F8: scale slots (by tile parity)
+  static constexpr int CONV = F8 ? NL : 0;             // F8: "slot converted" barriers
+  static constexpr int OFF_SCALE = OFF_LAT + NL * LAT_SLOT;
+  static constexpr int OFF_BAR = OFF_SCALE + NSC * SC_SLOT;
+  static constexpr int N_BAR = 2 * NL + 2 * NR + 1 + 2 + 2 + 2 + 2 + 1 + CONV + 2 * NSC;
   static constexpr int OFF_RED = OFF_BAR + N_BAR * 8 + 16;
   static constexpr int SMEM = OFF_RED + 2 * 4 * H * 4 + 1024;
   static constexpr int TMEM_COLS = 6 * H <= 128 ? 128 : 256;
   static constexpr uint32_t P_LAYOUT = H == 16 ? SW32 : SW64;
-  static_assert(OFF_P % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_LAT % 1024 == 0, "1 KB alignment");
+  static_assert(OFF_P % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_LAT % 1024 == 0 && OFF_SCALE % 1024 == 0,
+                "1 KB alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -314,11 +322,16 @@ __global__ void mla_attn_plan_kernel(const int32_t* __restrict__ kv_len, const i
   if (tid == 0) *n_units = n;
 }
 
-template <int H>
-__global__ void __launch_bounds__(ATT_THREADS, 1)
+// m_cache: bf16 rows as {value, slot, block} (64 x 64 boxes); F8: the rows'
+// bytes as {byte, slot, block} (128-byte x 64 boxes of codes, no swizzle),
+// with m_rope8 (bf16 view of the same rows, k^R boxes) and m_scale8 (16-byte
+// x 64 boxes of the scales).
+template <int H, bool F8>
+__global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
     mla_attn_kernel(const __grid_constant__ CUtensorMap m_qlat, const __grid_constant__ CUtensorMap m_qrope,
-                    const __grid_constant__ CUtensorMap m_cache, const AttnArgs a) {
-  using C = AttnCfg<H>;
+                    const __grid_constant__ CUtensorMap m_cache, const __grid_constant__ CUtensorMap m_rope8,
+                    const __grid_constant__ CUtensorMap m_scale8, const AttnArgs a) {
+  using C = AttnCfg<H, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -333,7 +346,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* p_full = s_free + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* grp_bar = pv_done + 2;  // 128-thread barrier of the softmax warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(grp_bar + 1);
+  uint64_t* lat_conv = grp_bar + 1;  // F8: latent slot converted to bf16 (128 converter arrivals)
+  uint64_t* sc_full = lat_conv + C::CONV;
+  uint64_t* sc_empty = sc_full + C::NSC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sc_empty + C::NSC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][H]
 
@@ -361,6 +377,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       mbar_init(&pv_done[i], 1);
     }
     mbar_init(grp_bar, 128);
+    for (int i = 0; i < C::CONV; ++i) mbar_init(&lat_conv[i], 128);
+    for (int i = 0; i < C::NSC; ++i) {
+      mbar_init(&sc_full[i], 1);
+      mbar_init(&sc_empty[i], 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -395,7 +416,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       };
       // Pages are prefetched into L2 ATT_PREFETCH tiles ahead of their TMA
       // loads, which then see L2 rather than HBM latency.
-      constexpr uint32_t PAGE_BYTES = 64u * (ATT_DC + ATT_DR) * 2u;
+      constexpr uint32_t PAGE_BYTES = 64u * (F8 ? fp8_row_bytes(ATT_DC, ATT_DR) : (ATT_DC + ATT_DR) * 2);
       TileCursor c, cf;
       c.init(a, range);
       cf = c;
@@ -425,11 +446,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         prefetch();
         int blk[2];
         for (int p = 0; p < 2; ++p) blk[p] = page_block(c, c.tok() / 64 + p);
+        if (F8) {
+          // the rows' scales, read by the converter warps first
+          const int ss = g % 2;
+          if (g >= 2 && !mbar_wait(&sc_empty[ss], ((g / 2) - 1) & 1, abort_flag, 406)) break;
+          uint8_t* sdst = smem + C::OFF_SCALE + ss * C::SC_SLOT;
+          mbar_expect_tx(&sc_full[ss], C::SC_SLOT);
+          for (int p = 0; p < 2; ++p)
+            tma_load_3d(sdst + p * 1024, &m_scale8, &sc_full[ss], fp8_scale_off(ATT_DC, ATT_DR), 0, blk[p]);
+        }
         const int rs = g % C::NR;
         if (g >= C::NR && !mbar_wait(&rope_empty[rs], ((g / C::NR) - 1) & 1, abort_flag, 404)) break;
         uint8_t* rdst = smem + C::OFF_ROPE + rs * C::ROPE_SLOT;
         mbar_expect_tx(&rope_full[rs], C::ROPE_SLOT);
-        for (int p = 0; p < 2; ++p) tma_load_3d(rdst + p * 8192, &m_cache, &rope_full[rs], ATT_DC, 0, blk[p]);
+        for (int p = 0; p < 2; ++p)
+          tma_load_3d(rdst + p * 8192, F8 ? &m_rope8 : &m_cache, &rope_full[rs], F8 ? ATT_DC / 2 : ATT_DC, 0, blk[p]);
         for (int m = 0; m < 4; ++m) {
           const int li = 4 * g + m;  // latent slot uses so far
           const int s = li % C::NL;
@@ -438,10 +469,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             break;
           }
           uint8_t* dst = smem + C::OFF_LAT + s * C::LAT_SLOT;
-          mbar_expect_tx(&lat_full[s], C::LAT_SLOT);
-          for (int hh = 0; hh < 2; ++hh)
-            for (int p = 0; p < 2; ++p)
-              tma_load_3d(dst + hh * 16384 + p * 8192, &m_cache, &lat_full[s], m * 128 + hh * 64, 0, blk[p]);
+          if (F8) {
+            // the codes of latent columns [128 m, 128 m + 128) of both pages
+            // land in the slot's upper half, where the converters expand them
+            mbar_expect_tx(&lat_full[s], C::LAT_SLOT / 2);
+            for (int p = 0; p < 2; ++p) tma_load_3d(dst + 16384 + p * 8192, &m_cache, &lat_full[s], m * 128, 0, blk[p]);
+          } else {
+            mbar_expect_tx(&lat_full[s], C::LAT_SLOT);
+            for (int hh = 0; hh < 2; ++hh)
+              for (int p = 0; p < 2; ++p)
+                tma_load_3d(dst + hh * 16384 + p * 8192, &m_cache, &lat_full[s], m * 128 + hh * 64, 0, blk[p]);
+          }
         }
         c.step(a);
       }
@@ -508,7 +546,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
               const int c = kq - 1;
               const int li = jq * 4 + c / 2;
               const int s = li % C::NL;
-              ready = (c & 1) || mbar_test(smem_u32(&lat_full[s]), (li / C::NL) & 1);
+              ready = (c & 1) || mbar_test(smem_u32(F8 ? &lat_conv[s] : &lat_full[s]), (li / C::NL) & 1);
               ka = lat_base + s * C::LAT_SLOT + (c & 1) * 16384;
               qchunk = c;
             }
@@ -548,6 +586,61 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           }
         }
       }
+    }
+  } else if (F8 && warp >= 6) {
+    // ------------------------------------------------------------ F8 converters
+    // Thread = (page p, token row r) of every latent slot: it reads the
+    // row's 128 codes from the slot's upper half and writes them as bf16
+    // times the row's scale 2^e into both halves in the MMA's SW128 layout
+    // (codes of columns 0..63 -> the lower half, 64..127 -> the upper half,
+    // over exactly the bytes this thread just read, so no other thread's
+    // input is touched).
+    const int ct = threadIdx.x - ATT_THREADS;
+    const int p = ct >> 6, r = ct & 63;
+    TileCursor c;
+    c.init(a, range);
+    bool ok = true;
+    while (ok && !c.done()) {
+      const int g = c.g;
+      const int ss = g % 2;
+      if (!mbar_wait(&sc_full[ss], (g / 2) & 1, abort_flag, 431)) break;
+      const float scale = *reinterpret_cast<const float*>(smem + C::OFF_SCALE + ss * C::SC_SLOT + p * 1024 + r * 16);
+      mbar_arrive(&sc_empty[ss]);
+      // bf16 exponent rebase plus e for both halves (a zero-filled row past
+      // the cache has scale 0: any value, its codes are all zero)
+      const int e = (int)((__float_as_uint(scale) >> 23) & 0xFFu) - 127;
+      const uint32_t bias = ((uint32_t)(112 + e) & 0xFFu) << 7;
+      for (int m = 0; m < 4 && ok; ++m) {
+        const int li = 4 * g + m, s = li % C::NL;
+        if (!mbar_wait(&lat_full[s], (li / C::NL) & 1, abort_flag, 432)) {
+          ok = false;
+          break;
+        }
+        uint8_t* slot = smem + C::OFF_LAT + s * C::LAT_SLOT + p * 8192 + r * 128;
+        const uint4* in = reinterpret_cast<const uint4*>(slot + 16384);
+        uint4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = in[k];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          // codes 16k .. 16k+15: bf16 columns 16(k%4) .. +15 of half k/4, 16-byte units 2(k%4), 2(k%4)+1
+          uint8_t* half = slot + (k >> 2) * 16384;
+          const uint32_t u0 = 2u * (k & 3);
+          const uint4 lo = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[k].x, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[k].x >> 16), bias),
+                                      bf16x2_from_e4m3x2((uint16_t)v[k].y, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[k].y >> 16), bias));
+          const uint4 hi = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[k].z, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[k].z >> 16), bias),
+                                      bf16x2_from_e4m3x2((uint16_t)v[k].w, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[k].w >> 16), bias));
+          *reinterpret_cast<uint4*>(half + ((u0 ^ (uint32_t)(r & 7)) << 4)) = lo;
+          *reinterpret_cast<uint4*>(half + (((u0 + 1) ^ (uint32_t)(r & 7)) << 4)) = hi;
+        }
+        fence_proxy_async_smem();  // the tensor core reads what these threads wrote
+        mbar_arrive(&lat_conv[s]);
+      }
+      c.step(a);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue

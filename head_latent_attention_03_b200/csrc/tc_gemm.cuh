@@ -50,10 +50,11 @@ struct GemmEpi {
   int d_hr;
   // EPI_CACHE
   int d_c;
-  float* lat_f32;            // non-null: c^KV goes here ([t][d_c] fp32) for the latent RMSNorm, not to the cache
+  float* lat_f32;            // non-null: c^KV goes here ([t][d_c] fp32) for the second pass (latent
+                             // RMSNorm, FP8 encoding), not to the cache
   const int32_t* seq_idx;    // [T]
-  __nv_bfloat16* pool;
-  int num_blocks, max_blocks, block_size;
+  uint8_t* pool;             // rows of row_bytes; k^R (bf16) at byte rope_off of its row
+  int num_blocks, max_blocks, block_size, row_bytes, rope_off;
   const int32_t* table;
   // EPI_Q
   int nq, n_h;
@@ -117,7 +118,6 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
           __floats2bfloat162_rn(v.x, v.y);
       break;
     case EPI_CACHE: {
-      const int row = e.d_c + e.d_hr;
       const long long p = e.pos[t];
       if (n < e.d_c && e.lat_f32) {
         *reinterpret_cast<float2*>(e.lat_f32 + (long long)t * e.d_c + n) = v;
@@ -136,7 +136,8 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
         if (n == 0) record_error(ERR_CAPACITY, 301);
         break;
       }
-      __nv_bfloat16* dst = e.pool + ((long long)blk * e.block_size + p % e.block_size) * row + n;
+      uint8_t* rowp = e.pool + ((long long)blk * e.block_size + p % e.block_size) * e.row_bytes;
+      uint8_t* dst = n < e.d_c ? rowp + 2 * n : rowp + e.rope_off + 2 * (n - e.d_c);
       *reinterpret_cast<__nv_bfloat162*>(dst) = __floats2bfloat162_rn(v.x, v.y);
       break;
     }

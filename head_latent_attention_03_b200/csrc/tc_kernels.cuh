@@ -97,6 +97,35 @@ inline bool map_cache_chunks(CUtensorMap* m, const void* pool, int num_blocks, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// FP8 cache rows (row_bytes each) as bytes {byte, slot, block}; box = box_bytes
+// x 64 slots of one page, no swizzle (the codes of 128 latent columns, or a
+// row's 16-byte scale field).
+inline bool map_cache_bytes(CUtensorMap* m, const void* pool, int num_blocks, int row_bytes, uint32_t box_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)row_bytes, 64, (cuuint64_t)num_blocks};
+  cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * 64};
+  cuuint32_t box[3] = {box_bytes, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(pool), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The same FP8 rows as bf16 elements {value, slot, block} (row_bytes / 2
+// values per row): 64 x 64 boxes with the 128-byte swizzle, for k^R.
+inline bool map_cache_bf16_view(CUtensorMap* m, const void* pool, int num_blocks, int row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)row_bytes / 2, 64, (cuuint64_t)num_blocks};
+  cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)row_bytes * 64};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A row-major bf16 matrix (`rows` rows of `inner` elements, rows `row_bytes`
 // apart) as a 3D map {column in chunk, row, 64-column chunk}: a box of
 // box_rows rows x kc chunks lands chunk-major (each chunk box_rows x 128 B,
@@ -325,8 +354,14 @@ inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
 
 // Workspace of the projections: only the bf16 intermediates between two
 // GEMMs (K splits are reduced inside each GEMM's cluster).
+inline bool fp8_cache(const mla_layer_desc* D) { return D->cache_dtype == MLA_CACHE_FP8_E4M3; }
+// bytes of one cache row: [c^KV | k^R] in bf16, or the FP8 row (codes, bf16
+// k^R, scale, padding)
+inline int cache_row_bytes(const mla_layer_desc* D) {
+  return fp8_cache(D) ? fp8_row_bytes(D->d_c, D->d_hr) : (D->d_c + D->d_hr) * 2;
+}
 inline size_t ws_compress(const mla_layer_desc* D, int T) {
-  return D->latent_norm ? (size_t)T * D->d_c * 4 + 256 : 0;
+  return D->latent_norm || fp8_cache(D) ? (size_t)T * D->d_c * 4 + 256 : 0;
 }
 inline size_t ws_absorb(const mla_layer_desc* D, int T) {
   Carver c{nullptr, 0};
@@ -449,14 +484,14 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   if (!aligned16(h) || !aligned16(w->w_dkv) || !aligned16(w->w_kr) || !aligned16(cache->pool) ||
       (D->latent_norm && !aligned16(w->g_kv)))
     return MLA_ERR_INVALID_ARG;
-  float* lat = nullptr;  // fp32 c^KV for the latent RMSNorm
-  if (D->latent_norm) {
+  float* lat = nullptr;  // fp32 c^KV for the second pass (latent RMSNorm, FP8 encoding)
+  if (D->latent_norm || fp8_cache(D)) {
     Carver cv = carve(ws, ws_bytes);
     lat = (float*)cv.take((size_t)T * D->d_c * 4);
     if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   }
   // [c^KV ; k^R] = [W^DKV ; W^KR] h  (eq 9 + decoupled key), RoPE on k^R,
-  // bf16 rows scattered into the paged cache
+  // bf16 rows scattered into the paged cache (with the second pass: k^R only)
   GemmCall c{};
   c.a0 = w->w_dkv;
   c.rows0 = D->d_c;
@@ -476,29 +511,35 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   e.d_hr = D->d_hr;
   e.d_c = D->d_c;
   e.seq_idx = seq_idx;
-  e.pool = (__nv_bfloat16*)cache->pool;
+  e.pool = (uint8_t*)cache->pool;
   e.num_blocks = cache->num_blocks;
   e.max_blocks = cache->max_blocks;
   e.block_size = D->block_size;
+  e.row_bytes = cache_row_bytes(D);
+  e.rope_off = fp8_cache(D) ? D->d_c : 2 * D->d_c;
   e.table = cache->block_table;
   e.lat_f32 = lat;
   mla_status_t s = run_gemm(c, e, plan_compress(D, T), st);
   if (s != MLA_OK || !lat) return s;
-  // c^KV <- scale_kv * g_kv * c^KV / rms(c^KV), into the cache row
+  // c^KV <- scale_kv * g_kv * c^KV / rms(c^KV) (with the norm), into the
+  // cache row as bf16 or as E4M3 codes with the row's scale
   NormArgs na{};
   na.x = lat;
   na.n = D->d_c;
+  na.do_norm = D->latent_norm ? 1 : 0;
   na.gain = (const __nv_bfloat16*)w->g_kv;
   na.eps = (float)D->norm_eps;
   na.scale = (float)D->scale_kv;
-  na.pool = (__nv_bfloat16*)cache->pool;
+  na.pool = (uint8_t*)cache->pool;
   na.table = cache->block_table;
   na.seq_idx = seq_idx;
   na.pos = pos;
   na.num_blocks = cache->num_blocks;
   na.max_blocks = cache->max_blocks;
   na.block_size = D->block_size;
-  na.row = D->d_c + D->d_hr;
+  na.row_bytes = cache_row_bytes(D);
+  na.fp8 = fp8_cache(D) ? 1 : 0;
+  na.scale_off = fp8_scale_off(D->d_c, D->d_hr);
   return launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) == cudaSuccess ? MLA_OK
                                                                                                       : MLA_ERR_CUDA;
 }
@@ -547,6 +588,7 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
       NormArgs na{};
       na.x = cq32;
       na.n = D->d_cq;
+      na.do_norm = 1;
       na.gain = (const __nv_bfloat16*)w->g_q;
       na.eps = (float)D->norm_eps;
       na.scale = (float)D->scale_q;
@@ -776,12 +818,19 @@ static mla_status_t tc_prefill_unabsorbed(const mla_layer_desc* D, const mla_wei
 }
 
 template <int H>
-static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, const CUtensorMap& mc, const AttnArgs& a,
-                               dim3 grid, cudaStream_t st) {
-  auto kfn = mla_attn_kernel<H>;
-  constexpr int smem = AttnCfg<H>::SMEM;
+static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, const CUtensorMap& mc,
+                               const CUtensorMap& mr8, const CUtensorMap& ms8, bool f8, const AttnArgs& a, dim3 grid,
+                               cudaStream_t st) {
+  if (f8) {
+    auto kfn = mla_attn_kernel<H, true>;
+    constexpr int smem = AttnCfg<H, true>::SMEM;
+    cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return launch_pdl(kfn, grid, dim3(AttnCfg<H, true>::THREADS), smem, st, 1, mq, mr, mc, mr8, ms8, a);
+  }
+  auto kfn = mla_attn_kernel<H, false>;
+  constexpr int smem = AttnCfg<H, false>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  return launch_pdl(kfn, grid, dim3(ATT_THREADS), smem, st, 1, mq, mr, mc, a);
+  return launch_pdl(kfn, grid, dim3(AttnCfg<H, false>::THREADS), smem, st, 1, mq, mr, mc, mc, mc, a);
 }
 
 // kv_begin (partial decode): rows [kv_begin[b], kv_len[b]) only, every row
@@ -813,7 +862,17 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   CUtensorMap mq, mr, mc;
   bool ok = map_2d(&mq, q_lat, ATT_DC, (uint64_t)rows * D->n_h, ATT_DC * 2, 64, q_box);
   ok = ok && map_2d(&mr, q_rope, ATT_DR, (uint64_t)rows * D->n_h, ATT_DR * 2, 64, q_box);
-  ok = ok && map_cache(&mc, cache->pool, cache->num_blocks, ATT_DC + ATT_DR);
+  const bool f8 = fp8_cache(D);
+  CUtensorMap mr8, ms8;  // FP8 rows: k^R view and scales (m_cache: the codes)
+  if (f8) {
+    const int rb = cache_row_bytes(D);
+    ok = ok && map_cache_bytes(&mc, cache->pool, cache->num_blocks, rb, 128);
+    ok = ok && map_cache_bf16_view(&mr8, cache->pool, cache->num_blocks, rb);
+    ok = ok && map_cache_bytes(&ms8, cache->pool, cache->num_blocks, rb, 16);
+  } else {
+    ok = ok && map_cache(&mc, cache->pool, cache->num_blocks, ATT_DC + ATT_DR);
+    mr8 = ms8 = mc;
+  }
   if (!ok) return MLA_ERR_CUDA;
   AttnArgs a;
   a.n_h = D->n_h;
@@ -845,7 +904,8 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
     e = launch_pdl(mla_attn_pair_kernel, grid, dim3(PairCfg::THREADS), PairCfg::SMEM, st, 1, mq, mr, m1, m2, a);
   } else {
     dim3 grid(p.workers * attn_groups(D));
-    e = H == 16 ? launch_attn<16>(mq, mr, mc, a, grid, st) : launch_attn<32>(mq, mr, mc, a, grid, st);
+    e = H == 16 ? launch_attn<16>(mq, mr, mc, mr8, ms8, f8, a, grid, st)
+                : launch_attn<32>(mq, mr, mc, mr8, ms8, f8, a, grid, st);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
   if (p.max_slots > 0) {

@@ -99,6 +99,13 @@ class MLALayer:
         D, dev, dt = self.dims, self.device, torch_dtype(self.dims)
         new = batch.workload.new_tokens
         pool = to_device(batch.pool, dt, dev)
+        if getattr(D, "cache_dtype", "bf16") == "fp8":
+            # the drawn rows, encoded on the device into the FP8 row format
+            rows = pool
+            pool = torch.empty((rows.shape[0], rows.shape[1], mla.cache_row_bytes(self.desc)), dtype=torch.uint8,
+                               device=dev)
+            mla.cache_quantize(self.desc, rows, pool)
+            del rows
         table = torch.from_numpy(batch.block_table).to(dev)
         h = to_device(batch.h, dt, dev)
         seq_idx = torch.from_numpy(batch.seq_idx.astype(np.int32)).to(dev)

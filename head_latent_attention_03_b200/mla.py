@@ -15,6 +15,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmla_b200.so")
 
 MLA_F32, MLA_BF16 = 0, 1
+MLA_CACHE_NATIVE, MLA_CACHE_FP8_E4M3 = 0, 1
 STATUS = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED", 3: "MLA_ERR_CAPACITY",
           4: "MLA_ERR_CUDA", 5: "MLA_ERR_DEVICE_TIMEOUT"}
 
@@ -31,7 +32,7 @@ class LayerDesc(ctypes.Structure):
                 ("dtype", ctypes.c_int), ("rope_base", ctypes.c_double), ("yarn_scale", ctypes.c_double),
                 ("yarn_orig_ctx", ctypes.c_int), ("yarn_alpha", ctypes.c_double), ("yarn_beta", ctypes.c_double),
                 ("attn_logit_factor", ctypes.c_double), ("latent_norm", ctypes.c_int), ("norm_eps", ctypes.c_double),
-                ("scale_kv", ctypes.c_double), ("scale_q", ctypes.c_double)]
+                ("scale_kv", ctypes.c_double), ("scale_q", ctypes.c_double), ("cache_dtype", ctypes.c_int)]
 
 
 class Weights(ctypes.Structure):
@@ -91,6 +92,9 @@ _SIGS = {
                                                    ctypes.c_void_p]),
     "mla_out_proj_unabsorbed": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
+    "mla_cache_row_bytes": (ctypes.c_size_t, [ctypes.POINTER(LayerDesc)]),
+    "mla_cache_quantize": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.c_void_p, ctypes.c_longlong,
+                                          ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 
@@ -119,7 +123,8 @@ def layer_desc(dims) -> LayerDesc:
                      MLA_BF16 if dims.dtype == "bf16" else MLA_F32, dims.rope_base, dims.yarn_scale,
                      dims.yarn_orig_ctx, dims.yarn_alpha, dims.yarn_beta, dims.attn_logit_factor,
                      int(getattr(dims, "latent_norm", False)), getattr(dims, "norm_eps", 0.0),
-                     getattr(dims, "scale_kv", 1.0), getattr(dims, "scale_q", 1.0))
+                     getattr(dims, "scale_kv", 1.0), getattr(dims, "scale_q", 1.0),
+                     MLA_CACHE_FP8_E4M3 if getattr(dims, "cache_dtype", "bf16") == "fp8" else MLA_CACHE_NATIVE)
 
 
 def _ptr(t) -> Optional[int]:
@@ -153,6 +158,17 @@ def launch_count() -> int:
 
 def status_string(code: int) -> str:
     return lib().mla_status_string(code).decode()
+
+
+def cache_row_bytes(desc: LayerDesc) -> int:
+    return lib().mla_cache_row_bytes(ctypes.byref(desc))
+
+
+def cache_quantize(desc, src, dst, stream=None):
+    """bf16 cache rows src [..., d_c + d_hr] -> FP8 rows dst [..., cache_row_bytes] (uint8)."""
+    n = src.numel() // (desc.d_c + desc.d_hr)
+    _check("mla_cache_quantize", lib().mla_cache_quantize(ctypes.byref(desc), _ptr(src), n, _ptr(dst),
+                                                          _stream(stream)))
 
 
 def workspace_size(desc: LayerDesc, T: int, B: int, max_kv_len: int) -> int:

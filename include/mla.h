@@ -48,6 +48,10 @@
  *  MLA_BF16 (tcgen05 tensor-core kernels): block_size == 64, d_c == 512,
  *    d_hr == 64, d_h % 64 == 0, d % 64 == 0, d_cq % 64 == 0, n_h in {16, 32,
  *    64, 128}.
+ *  MLA_CACHE_FP8_E4M3: MLA_BF16 layers; the latent attention
+ *    (mla_decode_attn, mla_decode_attn_noalloc, mla_decode_attn_partial,
+ *    mla_prefill_attn) reads FP8 rows for n_h in {16, 32, 64}; n_h = 128 and
+ *    the un-absorbed prefill return MLA_ERR_UNSUPPORTED.
  */
 #ifndef MLA_H
 #define MLA_H
@@ -69,6 +73,12 @@ typedef enum {
 } mla_status_t;
 
 typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype_t;
+
+/* Storage of the latent cache rows (mla_layer_desc.cache_dtype). */
+typedef enum {
+  MLA_CACHE_NATIVE = 0,   /* [c^KV | k^R] in the layer's element type */
+  MLA_CACHE_FP8_E4M3 = 1  /* FP8 rows, MLA_BF16 layers only (see mla_paged_cache) */
+} mla_cache_dtype_t;
 
 /* Layer description, in the pages' notation. */
 typedef struct {
@@ -93,6 +103,10 @@ typedef struct {
   int latent_norm;
   double norm_eps;           /* >= 0 */
   double scale_kv, scale_q;  /* > 0 */
+  /* mla_cache_dtype_t.  The KV cache is quantised for serving (DeepSeek-V2
+   * explainer, section 3.1.4); MLA_CACHE_FP8_E4M3 stores c^KV as FP8 codes
+   * with one power-of-two scale per row and keeps k^R in bf16. */
+  int cache_dtype;
 } mla_layer_desc;
 
 /* Projection matrices, [out, in] row-major, element type = desc.dtype.
@@ -107,16 +121,37 @@ typedef struct {
   const void *g_kv, *g_q;
 } mla_weights;
 
-/* Paged latent cache: pool [num_blocks, block_size, d_c + d_hr]; token j of
+/* Paged latent cache: pool [num_blocks, block_size, row]; token j of
  * sequence b lives at pool[block_table[b*max_blocks + j/block_size]][j % block_size].
  * Slots that no sequence has written may hold any bits (NaN included): the
- * attention kernels never let them reach a result. */
+ * attention kernels never let them reach a result.
+ * Row (mla_cache_row_bytes bytes):
+ *   MLA_CACHE_NATIVE    [c^KV (d_c) | k^R (d_hr)] in the layer's element type
+ *   MLA_CACHE_FP8_E4M3  bytes [0, d_c)               E4M3 codes q of c^KV
+ *                       bytes [d_c, d_c + 2 d_hr)    k^R, bf16
+ *                       bytes [d_c + 2 d_hr, +4)     fp32 scale 2^e
+ *                       zero padding to a multiple of 16 bytes (656 bytes at
+ *                       d_c = 512, d_hr = 64)
+ *     c^KV = q * 2^e, E4M3 = OCP 8-bit float (sign, 4 exponent bits with bias
+ *     7, 3 mantissa bits, subnormals, largest finite 448); e is the smallest
+ *     integer with max|c^KV| <= 448 * 2^e, codes are rounded to nearest even
+ *     and saturated.  The attention multiplies with c^KV = q * 2^e exactly. */
 typedef struct {
   void* pool;
   int num_blocks;
   const int32_t* block_table;  /* [B, max_blocks] int32 */
   int max_blocks;
 } mla_paged_cache;
+
+/* Bytes of one cache row of this layer (0 for an invalid desc). */
+size_t mla_cache_row_bytes(const mla_layer_desc* desc);
+
+/* Encode n bf16 cache rows [n, d_c + d_hr] (e.g. a whole pool of
+ * num_blocks * block_size rows) as FP8 rows [n, mla_cache_row_bytes] in the
+ * format above; desc.cache_dtype must be MLA_CACHE_FP8_E4M3.  A NaN element
+ * (an unwritten slot) becomes a NaN code and is left out of its row's
+ * maximum.  src and dst must not overlap. */
+mla_status_t mla_cache_quantize(const mla_layer_desc* desc, const void* src, long long n, void* dst, void* stream);
 
 /* Bytes of scratch that every call below needs for T tokens per projection
  * call and B sequences of at most max_kv_len cached tokens per attention call

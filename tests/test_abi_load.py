@@ -58,6 +58,26 @@ def test_invalid_arguments_are_rejected_without_a_gpu(lib):
     assert mla.workspace_size(bad, 1, 1, 64) == 0
 
 
+def test_fp8_cache_rows_and_limits_without_a_gpu(lib):
+    import dataclasses
+    assert mla.cache_row_bytes(mla.layer_desc(LITE)) == 1152
+    assert mla.cache_row_bytes(mla.layer_desc(TINY)) == (TINY.d_c + TINY.d_hr) * 4
+    fp8 = mla.layer_desc(dataclasses.replace(LITE, cache_dtype="fp8"))
+    # 512 code bytes + 128 bytes of bf16 k^R + 4-byte scale, padded to 16 bytes
+    assert mla.cache_row_bytes(fp8) == 656
+    # FP8 rows need a bf16 layer: an fp32 layer with them is an invalid desc
+    assert mla.cache_row_bytes(mla.layer_desc(dataclasses.replace(TINY, cache_dtype="fp8"))) == 0
+    # the 128-head CTA-pair attention reads bf16 rows only: refused on the
+    # host, before any CUDA call (the pointers are never dereferenced)
+    v2 = mla.layer_desc(dataclasses.replace(V2, cache_dtype="fp8"))
+    cache = mla.PagedCache(16, 1, 16, 1)
+    code = mla.lib().mla_decode_attn(ctypes.byref(v2), 16, 16, ctypes.byref(cache), 16, 1, 16, 1 << 20, 0, 16,
+                                     None, None)
+    assert code == 2
+    # encoding rows into the FP8 format needs a desc with FP8 rows
+    assert mla.lib().mla_cache_quantize(ctypes.byref(mla.layer_desc(LITE)), 16, 1, 32, None) == 1
+
+
 def declared_arity():
     """Number of parameters of every function include/mla.h declares."""
     src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)

@@ -18,7 +18,7 @@ from head_latent_attention_03_b200 import inputs as I
 from head_latent_attention_03_b200 import mla
 from head_latent_attention_03_b200.layer import MLALayer
 from oracle import mla_oracle as O
-from tests.metrics import assert_bf16, assert_fp32, rms_rel, max_abs
+from tests.metrics import assert_bf16, assert_fp32, rms_rel, max_abs, check_fp8_row, decode_fp8_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -48,8 +48,9 @@ def np32(t):
 
 
 def new_rows(st, batch):
+    """The rows the step appended, as stored (FP8 cache: the raw bytes)."""
     D = batch.workload.dims
-    pool = np32(st.pool)
+    pool = st.pool.cpu().numpy() if st.pool.dtype == torch.uint8 else np32(st.pool)
     out = []
     for b, L in enumerate(batch.prior_len):
         for t in range(batch.workload.new_tokens):
@@ -73,7 +74,11 @@ def check_decode(w, seqs=None, num_splits=0, batch=None):
     ref = O.decode_batch(batch, weights_for(w), seqs=seqs, absorbed=True)
     ref_un = O.decode_batch(batch, weights_for(w), seqs=seqs, absorbed=False)
     rows = new_rows(st, batch)[seqs]
-    compare("cache row", rows, np.stack([r["row"] for r in ref]), D)
+    if D.cache_dtype == "fp8":
+        for i, r in enumerate(ref):
+            check_fp8_row(rows[i], r["row"], D.d_c, D.d_hr, O.e4m3_round, O.fp8_scale_exponent, f"cache row {i}")
+    else:
+        compare("cache row", rows, np.stack([r["row"] for r in ref]), D)
     compare("q_lat", np32(st.q_lat)[seqs], np.stack([r["q_lat"] for r in ref]), D)
     compare("q_rope", np32(st.q_rope)[seqs], np.stack([r["q_r"] for r in ref]), D)
     compare("o_lat", np32(st.o_lat)[seqs], np.stack([r["o_lat"] for r in ref]), D)
@@ -387,3 +392,81 @@ def test_unabsorbed_prefill_full_size_sampled():
     batch = I.gen_batch(w)
     layer, st = _unabsorbed(w, batch)
     _check_unabsorbed(w, batch, st, [(5, [0, 1, 127, 128, 2047, 4095]), (0, [63, 64, 4094])])
+
+
+# ----------------------------------------------------------------------------
+# FP8 latent cache (E4M3 codes of c^KV, one power-of-two scale per row, bf16
+# k^R): the encoding of the drawn rows is exact, the new row's codes follow
+# the oracle's rounding, and the attention over the dequantised rows matches
+# the oracle's attention over its own dequantised rows.
+# ----------------------------------------------------------------------------
+LITE_FP8_SMALL = dataclasses.replace(I.WORKLOADS["lite_fp8"], name="lite_fp8_small", batch=4,
+                                     prior="list:63,200,700,1500")
+
+
+def test_fp8_encoding_of_the_drawn_rows_is_exact():
+    w = LITE_FP8_SMALL
+    D = w.dims
+    batch = I.gen_batch(w)
+    layer = MLALayer(D, weights_for(w))
+    st = layer.upload(batch)
+    torch.cuda.synchronize()
+    assert mla.get_last_error() == 0
+    assert st.pool.shape[2] == mla.cache_row_bytes(layer.desc) == 656
+    raw = st.pool.cpu().numpy()
+    for b in range(w.batch):
+        L = int(batch.prior_len[b])
+        rows = O.gather_rows(batch.pool, batch.block_table[b], L, D.block_size)
+        got = np.stack([raw[batch.block_table[b, j // 64], j % 64] for j in range(L)])
+        codes, scale, k_r, pad = decode_fp8_rows(got, D.d_c, D.d_hr)
+        for j in range(L):
+            want, e = O.quantize_latent(rows[j, :D.d_c])
+            assert scale[j] == 2.0 ** e, (b, j)
+            assert np.array_equal(codes[j], want), (b, j)
+        assert np.array_equal(k_r, rows[:, D.d_c:])
+        assert not pad.any()
+
+
+@pytest.mark.parametrize("splits", [0, 3])
+def test_fp8_decode_small(splits):
+    check_decode(LITE_FP8_SMALL, num_splits=splits)
+
+
+@pytest.mark.parametrize("n_h", [32, 64])
+def test_fp8_decode_other_head_counts(n_h):
+    w = dataclasses.replace(LITE_FP8_SMALL, name=f"fp8_heads{n_h}",
+                            dims=dataclasses.replace(LITE_FP8_SMALL.dims, n_h=n_h))
+    check_decode(w)
+
+
+def test_fp8_decode_with_latent_norm():
+    # the normalised and scaled c^KV is what gets encoded
+    w = _with_norm(LITE_FP8_SMALL, "lite_fp8_norm")
+    check_decode(w)
+
+
+def test_fp8_full_size_sampled():
+    # 32 x 4096 prior tokens (the V2-Lite workload over an FP8 cache): two
+    # sequences through the oracle
+    w = I.WORKLOADS["lite_fp8"]
+    check_decode(w, seqs=[0, 31])
+
+
+def test_fp8_prefill_chunk():
+    # latent-form causal prefill over FP8 rows: 9 new tokens per sequence
+    w = dataclasses.replace(LITE_FP8_SMALL, name="lite_fp8_prefill", batch=2, prior="list:63,200", new_tokens=9)
+    batch = I.gen_batch(w)
+    layer, st = run_gpu(w, batch)
+    D, W = w.dims, weights_for(w)
+    rows_g = new_rows(st, batch)
+    for b in range(2):
+        L = int(batch.prior_len[b])
+        prior = O.gather_rows(batch.pool, batch.block_table[b], L, D.block_size)
+        new_r, outs = O.prefill_sequence(D, W, batch.h[b * 9:(b + 1) * 9], L, prior, [0, 4, 8], absorbed=True)
+        for q in range(9):
+            check_fp8_row(rows_g[b * 9 + q], new_r[q], D.d_c, D.d_hr, O.e4m3_round, O.fp8_scale_exponent,
+                          f"row {b},{q}")
+        for q in (0, 4, 8):
+            r = b * 9 + q
+            assert_bf16(np32(st.o_lat)[r], outs[q]["o_lat"], f"o_lat {b},{q}")
+            assert_bf16(np32(st.u)[r], outs[q]["u"], f"u {b},{q}")

@@ -34,6 +34,9 @@ CASES = [
     # wave (74 CTA pairs) needs more than the 32 MiB array, so the entry point
     # plans for fewer pairs (test_v2_batch64_plan_exceeds_the_array)
     (dataclasses.replace(I.WORKLOADS["v2"], name="v2_b64_auto"), 0),
+    # FP8 cache rows, automatic and explicit splits
+    (dataclasses.replace(I.WORKLOADS["lite_fp8"], name="lite_fp8_auto", batch=4, prior="list:300,1500,900,64"), 0),
+    (dataclasses.replace(I.WORKLOADS["lite_fp8"], name="lite_fp8_splits2", batch=4, prior="list:300,1500,900,64"), 2),
 ]
 
 
