@@ -2,7 +2,7 @@
 """Benchmark of the MLA decode layer step on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload v2|lite|long|prefill] [--no-cpu-baseline] [--no-extra]
+                    [--workload v2|lite|lite_fp8|long|prefill] [--no-cpu-baseline] [--no-extra]
 
 A step is one pass of the whole hot path over one batch: compress_append ->
 absorb_q -> decode attention (+ LSE combine) -> out_proj, through the C ABI.
@@ -43,6 +43,8 @@ WORKLOAD_TEXT = {
           "decode batch 64, prior cache lengths uniform in [1,8192], block 64, permuted page table",
     "lite": "DeepSeek-V2-Lite-shaped MLA layer (d=2048, n_h=16, d_h=128, d_c=512, d_h^R=64), bf16, "
             "decode batch 32, 4096 prior tokens each, block 64",
+    "lite_fp8": "the V2-Lite workload over an FP8 latent cache (E4M3 codes of c^KV with a power-of-two scale "
+                "per row, bf16 k^R: 656 bytes per token), bf16 compute",
     "long": "V2-shaped MLA layer, bf16, decode batch 4 over 131072 prior tokens each, YaRN s=40, split-KV",
     "prefill": "V2-shaped MLA layer, bf16, chunked prefill: 8 sequences x 4096 new tokens over 4096 cached",
 }
@@ -144,10 +146,18 @@ def committed_traffic(workload: str):
 # ---------------------------------------------------------------------------
 # work accounting (algorithmic, per attention launch)
 # ---------------------------------------------------------------------------
+def cache_row_bytes(dims) -> int:
+    """Bytes of one cached row: [c^KV | k^R] in bf16 (1152 at d_c 512, d_h^R 64),
+    or the FP8 row (E4M3 codes, bf16 k^R, fp32 scale, padded to 16 bytes: 656)."""
+    if getattr(dims, "cache_dtype", "bf16") == "fp8":
+        return (dims.d_c + 2 * dims.d_hr + 4 + 15) // 16 * 16
+    return dims.row * 2
+
+
 def attention_work(dims, kv_len, rows):
     """Bytes that must move and FLOPs of one attention launch (absorbed form)."""
     tok = int(sum(kv_len))
-    bytes_ = tok * dims.row * 2 + rows * dims.n_h * dims.row * 2 + rows * dims.n_h * dims.d_c * 2
+    bytes_ = tok * cache_row_bytes(dims) + rows * dims.n_h * dims.row * 2 + rows * dims.n_h * dims.d_c * 2
     flops = tok * 2 * dims.n_h * (2 * dims.d_c + dims.d_hr)
     return bytes_, flops
 
@@ -333,7 +343,7 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
 
 
 # Steps of the extra workloads (their steps are longer than the headline's).
-EXTRA_STEPS = {"lite": (100, 5), "long": (20, 3), "prefill": (2, 1)}
+EXTRA_STEPS = {"lite": (100, 5), "lite_fp8": (100, 5), "long": (20, 3), "prefill": (2, 1)}
 
 
 # ---------------------------------------------------------------------------
@@ -464,7 +474,7 @@ def run_ours(args):
     if not args.no_extra and not args.profile_run:
         del layer, st
         torch.cuda.empty_cache()
-        for name in ("lite", "long", "prefill"):
+        for name in ("lite", "lite_fp8", "long", "prefill"):
             if name != args.workload:
                 k, wu = EXTRA_STEPS[name]
                 extra[name] = measure_extra(name, k, wu, dev, peaks, peak_src)
@@ -563,7 +573,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["v2", "lite", "long", "prefill"], default="v2")
+    ap.add_argument("--workload", choices=["v2", "lite", "lite_fp8", "long", "prefill"], default="v2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--profile-run", action="store_true",

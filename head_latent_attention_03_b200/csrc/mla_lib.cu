@@ -216,6 +216,22 @@ mla_status_t mla_absorb_q(const mla_layer_desc* D, const mla_weights* w, const v
   return tc_absorb_q(D, w, h, pos, T, q_lat, q_rope, ws, ws_bytes, as_stream(stream));
 }
 
+mla_status_t mla_compress_append_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h,
+                                          const int32_t* seq_idx, const int32_t* pos, int T, mla_paged_cache* cache,
+                                          void* q_lat, void* q_rope, void* ws, size_t ws_bytes, void* stream) {
+  if (!desc_valid(D) || !w || !w->w_dkv || !w->w_kr || !w->w_uq || !w->w_qr || !w->w_uk || (D->d_cq && !w->w_dq) ||
+      !h || !seq_idx || !pos || T < 0 || !cache_valid(cache) || !q_lat || !q_rope ||
+      (D->latent_norm && (!w->g_kv || (D->d_cq && !w->g_q))))
+    return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (D->dtype == MLA_F32) {
+    const mla_status_t s = mla_compress_append(D, w, h, seq_idx, pos, T, cache, ws, ws_bytes, stream);
+    return s != MLA_OK ? s : mla_absorb_q(D, w, h, pos, T, q_lat, q_rope, ws, ws_bytes, stream);
+  }
+  if (!bf16_supported(D)) return MLA_ERR_UNSUPPORTED;
+  return tc_compress_absorb(D, w, h, seq_idx, pos, T, cache, q_lat, q_rope, ws, ws_bytes, as_stream(stream));
+}
+
 static mla_status_t f32_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
                                   const mla_paged_cache* cache, const int32_t* kv_len, const int32_t* q_start,
                                   int q_per_seq, int rows, void* ws, size_t ws_bytes, void* o_lat, float* lse,

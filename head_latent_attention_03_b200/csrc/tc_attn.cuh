@@ -618,22 +618,25 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
         }
         uint8_t* slot = smem + C::OFF_LAT + s * C::LAT_SLOT + p * 8192 + r * 128;
         const uint4* in = reinterpret_cast<const uint4*>(slot + 16384);
+        // thread r takes its row's 16-byte chunks in the order r, r+1, ...
+        // (mod 8), so the 32 rows of a warp spread over all banks
         uint4 v[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = in[k];
+        for (int j = 0; j < 8; ++j) v[j] = in[(j + r) & 7];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int j = 0; j < 8; ++j) {
           // codes 16k .. 16k+15: bf16 columns 16(k%4) .. +15 of half k/4, 16-byte units 2(k%4), 2(k%4)+1
+          const int k = (j + r) & 7;
           uint8_t* half = slot + (k >> 2) * 16384;
           const uint32_t u0 = 2u * (k & 3);
-          const uint4 lo = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[k].x, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[k].x >> 16), bias),
-                                      bf16x2_from_e4m3x2((uint16_t)v[k].y, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[k].y >> 16), bias));
-          const uint4 hi = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[k].z, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[k].z >> 16), bias),
-                                      bf16x2_from_e4m3x2((uint16_t)v[k].w, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[k].w >> 16), bias));
+          const uint4 lo = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[j].x, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[j].x >> 16), bias),
+                                      bf16x2_from_e4m3x2((uint16_t)v[j].y, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[j].y >> 16), bias));
+          const uint4 hi = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[j].z, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[j].z >> 16), bias),
+                                      bf16x2_from_e4m3x2((uint16_t)v[j].w, bias),
+                                      bf16x2_from_e4m3x2((uint16_t)(v[j].w >> 16), bias));
           *reinterpret_cast<uint4*>(half + ((u0 ^ (uint32_t)(r & 7)) << 4)) = lo;
           *reinterpret_cast<uint4*>(half + (((u0 + 1) ^ (uint32_t)(r & 7)) << 4)) = hi;
         }

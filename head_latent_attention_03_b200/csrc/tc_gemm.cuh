@@ -25,8 +25,10 @@
 // of the first weight tiles overlap the previous kernel of the step; every
 // load into shared memory and every output store waits for it.
 // A is K-major ([n][k] rows) or, for the per-head absorbed W^UK, MN-major
-// (memory [k][n], n contiguous).  Two weight segments (e.g. W^DKV and W^KR)
-// can share one launch: M tiles below m_tiles0 read map A0, the rest A1.
+// (memory [k][n], n contiguous).  Up to three weight segments that multiply
+// the same activations (e.g. W^DKV, W^KR and W^DQ, all applied to h) share one
+// launch: M tiles below m_tiles0 read map A0, the next m_tiles1 map A1, the
+// rest A2; the epilogue sees the features of the segments one after another.
 #pragma once
 
 #include "common.cuh"
@@ -37,7 +39,8 @@ namespace mla {
 enum GemmEpiKind : int {
   EPI_F32 = 0,    // fp32 y[z][t][n]
   EPI_BF16 = 1,   // bf16 y[z][t][n]
-  EPI_CACHE = 2,  // features [0, d_c): c^KV; [d_c, d_c + d_hr): RoPE_pos(k^R); bf16 into the paged cache
+  EPI_CACHE = 2,  // features [0, d_c): c^KV; [d_c, d_c + d_hr): RoPE_pos(k^R); bf16 into the paged cache;
+                  // [d_c + d_hr, d_c + d_hr + d_cq): c^Q (bf16 or fp32 [t][d_cq]) when W^DQ shares the launch
   EPI_Q = 3,      // features [0, nq): q^C (bf16 [t][nq]); [nq, nq + n_h d_hr): RoPE_pos(q^R) (bf16)
 };
 
@@ -56,6 +59,8 @@ struct GemmEpi {
   uint8_t* pool;             // rows of row_bytes; k^R (bf16) at byte rope_off of its row
   int num_blocks, max_blocks, block_size, row_bytes, rope_off;
   const int32_t* table;
+  void* cq_out;              // c^Q of the W^DQ segment: bf16, or fp32 when cq_f32
+  int cq_f32, d_cq;
   // EPI_Q
   int nq, n_h;
   __nv_bfloat16* q_c;
@@ -66,8 +71,8 @@ struct GemmArgs {
   int k_chunks;        // K / 64 (whole contraction)
   int k_chunks_split;  // chunks per split
   int splits;          // CTAs per cluster (K splits of one tile)
-  int m_tiles0;        // M tiles of segment 0
-  int n_out0, n_out1;  // rows of segment 0 / segment 1 (n_out1 = 0: one segment)
+  int m_tiles0, m_tiles1;      // M tiles of segments 0 and 1 (segment 2 has the rest)
+  int n_out0, n_out1, n_out2;  // rows of the segments (0: the segment is absent)
   int T;               // tokens
   int a_z_rows;        // per-batch row offset into A (K-major: output rows; MN-major: K rows)
   int b_z_cols;        // per-batch column offset into X
@@ -118,6 +123,15 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
           __floats2bfloat162_rn(v.x, v.y);
       break;
     case EPI_CACHE: {
+      if (n >= e.d_c + e.d_hr) {  // c^Q (eq 12), the W^DQ segment
+        const long long o = (long long)t * e.d_cq + (n - e.d_c - e.d_hr);
+        if (e.cq_f32)
+          *reinterpret_cast<float2*>(reinterpret_cast<float*>(e.cq_out) + o) = v;
+        else
+          *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(e.cq_out) + o) =
+              __floats2bfloat162_rn(v.x, v.y);
+        break;
+      }
       const long long p = e.pos[t];
       if (n < e.d_c && e.lat_f32) {
         *reinterpret_cast<float2*>(e.lat_f32 + (long long)t * e.d_c + n) = v;
@@ -164,6 +178,7 @@ __device__ __forceinline__ void gemm_epilogue(const GemmEpi& e, int z, int t, in
 template <int TN, bool A_MN, int KC, bool DEEP>
 __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_SM)
     gemm_bf16_kernel(const __grid_constant__ CUtensorMap mA0, const __grid_constant__ CUtensorMap mA1,
+                     const __grid_constant__ CUtensorMap mA2,
                      const __grid_constant__ CUtensorMap mB, const GemmArgs g) {
   using C = GemmCfg<TN, KC, DEEP>;
   static_assert(TN % 16 == 0 && TN >= 16 && TN <= 256, "token tile");
@@ -189,9 +204,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
     pdl_wait();
     if (g.b_tile_row[nt] < 0) nk = 0;
   }
-  const bool seg1 = mt >= g.m_tiles0;
-  const CUtensorMap* mA = seg1 ? &mA1 : &mA0;
-  const int m_row0 = (seg1 ? mt - g.m_tiles0 : mt) * GEMM_BM;  // first row inside the segment
+  const int seg = mt < g.m_tiles0 ? 0 : mt < g.m_tiles0 + g.m_tiles1 ? 1 : 2;
+  const CUtensorMap* mA = seg == 0 ? &mA0 : seg == 1 ? &mA1 : &mA2;
+  const int m_row0 = (mt - (seg == 0 ? 0 : seg == 1 ? g.m_tiles0 : g.m_tiles0 + g.m_tiles1)) * GEMM_BM;
+  const int n_base = seg == 0 ? 0 : seg == 1 ? g.n_out0 : g.n_out0 + g.n_out1;  // first feature of the segment
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
@@ -310,7 +326,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
   // this CTA's rows of the tile, summed over the cluster in rank order
   const int r0 = ((ks * GEMM_BM) / S) & ~1, r1 = ks == S - 1 ? GEMM_BM : (((ks + 1) * GEMM_BM) / S) & ~1;
   const int n_pairs = (r1 - r0) / 2;
-  const int n_seg = seg1 ? g.n_out1 : g.n_out0;
+  const int n_seg = seg == 0 ? g.n_out0 : seg == 1 ? g.n_out1 : g.n_out2;
   const uint32_t red_addr = smem_u32(red);
   if (ok) {
     // E elements per thread and round: all their S remote loads are issued
@@ -349,7 +365,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, GemmCfg<TN, KC, DEEP>::CTAS_PER_
             v.x += part[q][sr].x;
             v.y += part[q][sr].y;
           }
-        gemm_epilogue(g.e, z, t, (seg1 ? g.n_out0 : 0) + n_in_seg, v);
+        gemm_epilogue(g.e, z, t, n_base + n_in_seg, v);
       }
     }
   }

@@ -221,33 +221,35 @@ inline GemmPlan plan_gemm(int m_tiles, int Z, int T, int K, bool a_mn = false) {
 }
 
 template <int TN, bool A_MN, bool DEEP>
-inline cudaError_t launch_gemm_t(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B, const GemmArgs& g,
-                                 dim3 grid, cudaStream_t st) {
+inline cudaError_t launch_gemm_t(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& A2,
+                                 const CUtensorMap& B, const GemmArgs& g, dim3 grid, cudaStream_t st) {
   constexpr int KC = A_MN ? 1 : MLA_GEMM_KC;
   auto kfn = gemm_bf16_kernel<TN, A_MN, KC, DEEP>;
   constexpr int smem = GemmCfg<TN, KC, DEEP>::SMEM;
   cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  return launch_pdl(kfn, grid, dim3(GEMM_THREADS), smem, st, g.splits, A0, A1, B, g);
+  return launch_pdl(kfn, grid, dim3(GEMM_THREADS), smem, st, g.splits, A0, A1, A2, B, g);
 }
 
 template <bool A_MN, bool DEEP>
-inline cudaError_t launch_gemm_tn(int tn, const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& B,
-                                  const GemmArgs& g, dim3 grid, cudaStream_t st) {
+inline cudaError_t launch_gemm_tn(int tn, const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& A2,
+                                  const CUtensorMap& B, const GemmArgs& g, dim3 grid, cudaStream_t st) {
   switch (tn) {
-    case 32: return launch_gemm_t<32, A_MN, DEEP>(A0, A1, B, g, grid, st);
-    case 64: return launch_gemm_t<64, A_MN, DEEP>(A0, A1, B, g, grid, st);
-    case 128: return launch_gemm_t<128, A_MN, true>(A0, A1, B, g, grid, st);
-    default: return launch_gemm_t<256, A_MN, true>(A0, A1, B, g, grid, st);
+    case 32: return launch_gemm_t<32, A_MN, DEEP>(A0, A1, A2, B, g, grid, st);
+    case 64: return launch_gemm_t<64, A_MN, DEEP>(A0, A1, A2, B, g, grid, st);
+    case 128: return launch_gemm_t<128, A_MN, true>(A0, A1, A2, B, g, grid, st);
+    default: return launch_gemm_t<256, A_MN, true>(A0, A1, A2, B, g, grid, st);
   }
 }
 
-// One projection: Y = epilogue(A X) over two weight segments (rows0 of A0,
-// rows1 of A1), K contraction, Z batches.
+// One projection: Y = epilogue(A X) over up to three weight segments (rows0
+// of A0, rows1 of A1, rows2 of A2), K contraction, Z batches.
 struct GemmCall {
   const void* a0;
   int rows0;
   const void* a1;  // may be null
   int rows1;
+  const void* a2;  // may be null (only with a1)
+  int rows2;
   long long a_row_elems;  // row pitch of A in elements (K-major: K; MN-major: features)
   bool a_mn;              // A stored [k][n] (n contiguous)
   int a_mn_rows;          // MN-major: total K rows of the map (Z * K)
@@ -259,16 +261,21 @@ struct GemmCall {
 };
 
 inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan& p, cudaStream_t st) {
-  CUtensorMap A0, A1, B;
+  CUtensorMap A0, A1, A2, B;
   bool ok;
   const uint32_t kc = (uint32_t)gemm_kc(c.a_mn);
   if (!c.a_mn) {
     ok = map_rows_chunks(&A0, c.a0, (uint64_t)c.K, (uint64_t)c.rows0 * c.Z, (uint64_t)c.a_row_elems * 2, 128, kc);
     ok = ok && map_rows_chunks(&A1, c.a1 ? c.a1 : c.a0, (uint64_t)c.K, (uint64_t)(c.a1 ? c.rows1 : c.rows0) * c.Z,
                                (uint64_t)c.a_row_elems * 2, 128, kc);
+    if (c.a1 && c.a2)
+      ok = ok && map_rows_chunks(&A2, c.a2, (uint64_t)c.K, (uint64_t)c.rows2 * c.Z, (uint64_t)c.a_row_elems * 2, 128,
+                                 kc);
+    else
+      A2 = A0;
   } else {
     ok = map_2d(&A0, c.a0, (uint64_t)c.rows0, (uint64_t)c.a_mn_rows, (uint64_t)c.a_row_elems * 2, 64, 64);
-    A1 = A0;
+    A1 = A2 = A0;
   }
   ok = ok && map_rows_chunks(&B, c.x, (uint64_t)c.x_row_elems, (uint64_t)c.x_rows, (uint64_t)c.x_row_elems * 2,
                              (uint32_t)p.tn, kc);
@@ -278,22 +285,24 @@ inline mla_status_t run_gemm(const GemmCall& c, const GemmEpi& e, const GemmPlan
   g.k_chunks_split = p.kcs;
   g.splits = p.splits;
   g.m_tiles0 = (c.rows0 + GEMM_BM - 1) / GEMM_BM;
+  g.m_tiles1 = c.a1 ? (c.rows1 + GEMM_BM - 1) / GEMM_BM : 0;
   g.n_out0 = c.rows0;
   g.n_out1 = c.a1 ? c.rows1 : 0;
+  g.n_out2 = c.a1 && c.a2 ? c.rows2 : 0;
   g.T = c.T;
   g.a_z_rows = c.a_z_rows;
   g.b_z_cols = c.b_z_cols;
   g.b_tile_row = c.b_tile_row;
   g.e = e;
-  const int m_tiles = g.m_tiles0 + (c.a1 ? (c.rows1 + GEMM_BM - 1) / GEMM_BM : 0);
+  const int m_tiles = g.m_tiles0 + g.m_tiles1 + (g.n_out2 + GEMM_BM - 1) / GEMM_BM;
   dim3 grid(m_tiles * p.splits, c.b_tile_row ? c.n_tiles_override : p.n_tiles, c.Z);
   cudaError_t err;
   if (c.a_mn)
-    err = p.deep ? launch_gemm_tn<true, true>(p.tn, A0, A1, B, g, grid, st)
-                 : launch_gemm_tn<true, false>(p.tn, A0, A1, B, g, grid, st);
+    err = p.deep ? launch_gemm_tn<true, true>(p.tn, A0, A1, A2, B, g, grid, st)
+                 : launch_gemm_tn<true, false>(p.tn, A0, A1, A2, B, g, grid, st);
   else
-    err = p.deep ? launch_gemm_tn<false, true>(p.tn, A0, A1, B, g, grid, st)
-                 : launch_gemm_tn<false, false>(p.tn, A0, A1, B, g, grid, st);
+    err = p.deep ? launch_gemm_tn<false, true>(p.tn, A0, A1, A2, B, g, grid, st)
+                 : launch_gemm_tn<false, false>(p.tn, A0, A1, A2, B, g, grid, st);
   return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -311,15 +320,17 @@ inline mla_status_t run_gemm_paged(const GemmCall& c, const GemmEpi& e, const Ge
   g.k_chunks_split = p.kcs;
   g.splits = 1;
   g.m_tiles0 = (c.rows0 + GEMM_BM - 1) / GEMM_BM;
+  g.m_tiles1 = (c.rows1 + GEMM_BM - 1) / GEMM_BM;
   g.n_out0 = c.rows0;
   g.n_out1 = c.rows1;
+  g.n_out2 = 0;
   g.T = c.T;
   g.a_z_rows = 0;
   g.b_z_cols = 0;
   g.b_tile_row = c.b_tile_row;
   g.e = e;
   const int m_tiles = g.m_tiles0 + (c.rows1 + GEMM_BM - 1) / GEMM_BM;
-  const cudaError_t err = launch_gemm_t<64, false, false>(A0, A1, B, g, dim3(m_tiles, p.n_tiles, 1), st);
+  const cudaError_t err = launch_gemm_t<64, false, false>(A0, A1, A0, B, g, dim3(m_tiles, p.n_tiles, 1), st);
   return err == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -340,6 +351,9 @@ inline GemmPlan plan_compress(const mla_layer_desc* D, int T) {
   return plan_gemm((D->d_c + 127) / 128 + (D->d_hr + 127) / 128, 1, T, D->d);
 }
 inline GemmPlan plan_q1(const mla_layer_desc* D, int T) { return plan_gemm((D->d_cq + 127) / 128, 1, T, D->d); }
+inline GemmPlan plan_compress_q(const mla_layer_desc* D, int T) {
+  return plan_gemm((D->d_c + 127) / 128 + (D->d_hr + 127) / 128 + (D->d_cq + 127) / 128, 1, T, D->d);
+}
 inline GemmPlan plan_q2(const mla_layer_desc* D, int T) {
   const int q_in = D->d_cq ? D->d_cq : D->d;
   return plan_gemm((D->n_h * D->d_h + 127) / 128 + (D->n_h * D->d_hr + 127) / 128, 1, T, q_in);
@@ -366,8 +380,16 @@ inline size_t ws_compress(const mla_layer_desc* D, int T) {
 inline size_t ws_absorb(const mla_layer_desc* D, int T) {
   Carver c{nullptr, 0};
   if (D->d_cq) c.take((size_t)T * D->d_cq * 2);
-  if (D->d_cq && D->latent_norm) c.take((size_t)T * D->d_cq * 4);
   c.take((size_t)T * D->n_h * D->d_h * 2);
+  if (D->d_cq && D->latent_norm) c.take((size_t)T * D->d_cq * 4);
+  return c.used;
+}
+inline size_t ws_compress_absorb(const mla_layer_desc* D, int T) {
+  Carver c{nullptr, 0};
+  if (D->d_cq) c.take((size_t)T * D->d_cq * 2);
+  c.take((size_t)T * D->n_h * D->d_h * 2);
+  if (D->d_cq && D->latent_norm) c.take((size_t)T * D->d_cq * 4);
+  if (D->latent_norm || fp8_cache(D)) c.take((size_t)T * D->d_c * 4);
   return c.used;
 }
 inline size_t ws_out(const mla_layer_desc* D, int T) {
@@ -460,7 +482,7 @@ using namespace mla;
 
 static size_t tc_workspace_size(const mla_layer_desc* D, int T, int B, int max_kv_len) {
   size_t w = 0;
-  if (T > 0) w = std::max({ws_compress(D, T), ws_absorb(D, T), ws_out(D, T)});
+  if (T > 0) w = std::max({ws_compress(D, T), ws_absorb(D, T), ws_compress_absorb(D, T), ws_out(D, T)});
   if (B > 0 && max_kv_len > 0) {
     const int max_len = (max_kv_len + 63) / 64 * 64;
     // the automatic plan, or any explicit split count up to 16
@@ -476,6 +498,86 @@ static Carver carve(void* ws, size_t ws_bytes) {
   const uintptr_t a = (reinterpret_cast<uintptr_t>(b) + 255) & ~uintptr_t(255);
   const size_t lost = b ? a - reinterpret_cast<uintptr_t>(b) : 0;
   return Carver{b ? reinterpret_cast<uint8_t*>(a) : nullptr, ws_bytes > lost ? ws_bytes - lost : 0};
+}
+
+// Epilogue of the GEMM that writes new cache rows: [c^KV ; k^R] with RoPE on
+// k^R scattered into the paged cache, or (lat non-null) c^KV parked in fp32
+// for the second pass and only k^R written.
+static GemmEpi cache_epi(const mla_layer_desc* D, const int32_t* seq_idx, const int32_t* pos,
+                         const mla_paged_cache* cache, float* lat) {
+  GemmEpi e{};
+  e.kind = EPI_CACHE;
+  e.rope = rope_table(rope_of(D), D->d_hr);
+  e.pos = pos;
+  e.d_hr = D->d_hr;
+  e.d_c = D->d_c;
+  e.seq_idx = seq_idx;
+  e.pool = (uint8_t*)cache->pool;
+  e.num_blocks = cache->num_blocks;
+  e.max_blocks = cache->max_blocks;
+  e.block_size = D->block_size;
+  e.row_bytes = cache_row_bytes(D);
+  e.rope_off = fp8_cache(D) ? D->d_c : 2 * D->d_c;
+  e.table = cache->block_table;
+  e.lat_f32 = lat;
+  return e;
+}
+
+// Second pass over the parked fp32 c^KV: c^KV <- scale_kv * g_kv * c^KV /
+// rms(c^KV) (with the norm), into the cache row as bf16 or as E4M3 codes with
+// the row's scale.
+static mla_status_t kv_second_pass(const mla_layer_desc* D, const mla_weights* w, const float* lat,
+                                   const int32_t* seq_idx, const int32_t* pos, int T, const mla_paged_cache* cache,
+                                   cudaStream_t st) {
+  NormArgs na{};
+  na.x = lat;
+  na.n = D->d_c;
+  na.do_norm = D->latent_norm ? 1 : 0;
+  na.gain = (const __nv_bfloat16*)w->g_kv;
+  na.eps = (float)D->norm_eps;
+  na.scale = (float)D->scale_kv;
+  na.pool = (uint8_t*)cache->pool;
+  na.table = cache->block_table;
+  na.seq_idx = seq_idx;
+  na.pos = pos;
+  na.num_blocks = cache->num_blocks;
+  na.max_blocks = cache->max_blocks;
+  na.block_size = D->block_size;
+  na.row_bytes = cache_row_bytes(D);
+  na.fp8 = fp8_cache(D) ? 1 : 0;
+  na.scale_off = fp8_scale_off(D->d_c, D->d_hr);
+  return launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) == cudaSuccess ? MLA_OK
+                                                                                                      : MLA_ERR_CUDA;
+}
+
+// c^Q <- scale_q * g_q * c^Q / rms(c^Q), fp32 in, bf16 out.
+static mla_status_t cq_norm_pass(const mla_layer_desc* D, const mla_weights* w, const float* cq32, __nv_bfloat16* cq,
+                                 int T, cudaStream_t st) {
+  NormArgs na{};
+  na.x = cq32;
+  na.n = D->d_cq;
+  na.do_norm = 1;
+  na.gain = (const __nv_bfloat16*)w->g_q;
+  na.eps = (float)D->norm_eps;
+  na.scale = (float)D->scale_q;
+  na.out = cq;
+  na.out_t = D->d_cq;
+  return launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) == cudaSuccess ? MLA_OK
+                                                                                                      : MLA_ERR_CUDA;
+}
+
+// Scratch of the query path: c^Q (bf16), q^C, fp32 c^Q (latent norm) and, when
+// the append shares the first GEMM, the fp32 c^KV of the second pass.
+struct QueryWs {
+  __nv_bfloat16 *cq, *qc;
+  float *cq32, *lat;
+};
+static bool carve_queries(Carver& cv, const mla_layer_desc* D, int T, bool own_qc, bool with_lat, QueryWs* q) {
+  q->cq = D->d_cq ? (__nv_bfloat16*)cv.take((size_t)T * D->d_cq * 2) : nullptr;
+  q->qc = own_qc ? (__nv_bfloat16*)cv.take((size_t)T * D->n_h * D->d_h * 2) : nullptr;
+  q->cq32 = D->d_cq && D->latent_norm ? (float*)cv.take((size_t)T * D->d_cq * 4) : nullptr;
+  q->lat = with_lat && (D->latent_norm || fp8_cache(D)) ? (float*)cv.take((size_t)T * D->d_c * 4) : nullptr;
+  return cv.ok();
 }
 
 static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weights* w, const void* h,
@@ -504,102 +606,20 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   c.K = D->d;
   c.T = T;
   c.Z = 1;
-  GemmEpi e{};
-  e.kind = EPI_CACHE;
-  e.rope = rope_table(rope_of(D), D->d_hr);
-  e.pos = pos;
-  e.d_hr = D->d_hr;
-  e.d_c = D->d_c;
-  e.seq_idx = seq_idx;
-  e.pool = (uint8_t*)cache->pool;
-  e.num_blocks = cache->num_blocks;
-  e.max_blocks = cache->max_blocks;
-  e.block_size = D->block_size;
-  e.row_bytes = cache_row_bytes(D);
-  e.rope_off = fp8_cache(D) ? D->d_c : 2 * D->d_c;
-  e.table = cache->block_table;
-  e.lat_f32 = lat;
-  mla_status_t s = run_gemm(c, e, plan_compress(D, T), st);
+  mla_status_t s = run_gemm(c, cache_epi(D, seq_idx, pos, cache, lat), plan_compress(D, T), st);
   if (s != MLA_OK || !lat) return s;
-  // c^KV <- scale_kv * g_kv * c^KV / rms(c^KV) (with the norm), into the
-  // cache row as bf16 or as E4M3 codes with the row's scale
-  NormArgs na{};
-  na.x = lat;
-  na.n = D->d_c;
-  na.do_norm = D->latent_norm ? 1 : 0;
-  na.gain = (const __nv_bfloat16*)w->g_kv;
-  na.eps = (float)D->norm_eps;
-  na.scale = (float)D->scale_kv;
-  na.pool = (uint8_t*)cache->pool;
-  na.table = cache->block_table;
-  na.seq_idx = seq_idx;
-  na.pos = pos;
-  na.num_blocks = cache->num_blocks;
-  na.max_blocks = cache->max_blocks;
-  na.block_size = D->block_size;
-  na.row_bytes = cache_row_bytes(D);
-  na.fp8 = fp8_cache(D) ? 1 : 0;
-  na.scale_off = fp8_scale_off(D->d_c, D->d_hr);
-  return launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) == cudaSuccess ? MLA_OK
-                                                                                                      : MLA_ERR_CUDA;
+  return kv_second_pass(D, w, lat, seq_idx, pos, T, cache, st);
 }
 
-// q_c_out: write q^C [T, n_h, d_h] there (the un-absorbed prefill's queries);
-// q_lat may then be null (no W^UK absorption).
-static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos,
-                                int T, void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st,
-                                void* q_c_out = nullptr) {
-  if (!aligned16(h) || !aligned16(w->w_uq) || !aligned16(w->w_qr) || !aligned16(w->w_uk) ||
-      (D->d_cq && !aligned16(w->w_dq)) || !aligned16(q_lat) || !aligned16(q_rope) ||
-      (D->d_cq && D->latent_norm && !aligned16(w->g_q)))
-    return MLA_ERR_INVALID_ARG;
-  Carver cv = carve(ws, ws_bytes);
+// [q^C ; q^R] = [W^UQ ; W^QR] c^Q (eq 13 + decoupled query, RoPE on q^R), then
+// (q_lat non-null) q_lat_i = (W^UK_i)^T q^C_i.
+static mla_status_t queries_from_cq(const mla_layer_desc* D, const mla_weights* w, const void* qsrc,
+                                    const int32_t* pos, int T, __nv_bfloat16* qc, void* q_lat, void* q_rope,
+                                    cudaStream_t st) {
   const int nq = D->n_h * D->d_h, nr = D->n_h * D->d_hr;
   const int q_in = D->d_cq ? D->d_cq : D->d;
-  __nv_bfloat16* cq = D->d_cq ? (__nv_bfloat16*)cv.take((size_t)T * D->d_cq * 2) : nullptr;
-  __nv_bfloat16* qc = q_c_out ? (__nv_bfloat16*)q_c_out : (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
-  if (q_c_out && !aligned16(q_c_out)) return MLA_ERR_INVALID_ARG;
-  float* cq32 = D->d_cq && D->latent_norm ? (float*)cv.take((size_t)T * D->d_cq * 4) : nullptr;
-  if (!ws || !cv.ok()) return MLA_ERR_CAPACITY;
   mla_status_t s;
-  const void* qsrc = h;
-  if (D->d_cq) {  // c^Q = W^DQ h   (eq 12)
-    GemmCall c{};
-    c.a0 = w->w_dq;
-    c.rows0 = D->d_cq;
-    c.a_row_elems = D->d;
-    c.x = h;
-    c.x_rows = T;
-    c.x_row_elems = D->d;
-    c.K = D->d;
-    c.T = T;
-    c.Z = 1;
-    GemmEpi e{};
-    if (cq32) {  // fp32 c^Q, then the latent RMSNorm writes the bf16 c^Q
-      e.kind = EPI_F32;
-      e.out = cq32;
-    } else {
-      e.kind = EPI_BF16;
-      e.out = cq;
-    }
-    e.out_t = D->d_cq;
-    if ((s = run_gemm(c, e, plan_q1(D, T), st)) != MLA_OK) return s;
-    if (cq32) {
-      NormArgs na{};
-      na.x = cq32;
-      na.n = D->d_cq;
-      na.do_norm = 1;
-      na.gain = (const __nv_bfloat16*)w->g_q;
-      na.eps = (float)D->norm_eps;
-      na.scale = (float)D->scale_q;
-      na.out = cq;
-      na.out_t = D->d_cq;
-      if (launch_pdl(mla_latent_norm_kernel, dim3(T), dim3(NORM_THREADS), 0, st, 1, na) != cudaSuccess)
-        return MLA_ERR_CUDA;
-    }
-    qsrc = cq;
-  }
-  {  // [q^C ; q^R] = [W^UQ ; W^QR] c^Q   (eq 13 + decoupled query), RoPE on q^R
+  {
     GemmCall c{};
     c.a0 = w->w_uq;
     c.rows0 = nq;
@@ -647,6 +667,84 @@ static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, c
     if ((s = run_gemm(c, e, plan_q3(D, T), st)) != MLA_OK) return s;
   }
   return MLA_OK;
+}
+
+// q_c_out: write q^C [T, n_h, d_h] there (the un-absorbed prefill's queries);
+// q_lat may then be null (no W^UK absorption).
+static mla_status_t tc_absorb_q(const mla_layer_desc* D, const mla_weights* w, const void* h, const int32_t* pos,
+                                int T, void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st,
+                                void* q_c_out = nullptr) {
+  if (!aligned16(h) || !aligned16(w->w_uq) || !aligned16(w->w_qr) || !aligned16(w->w_uk) ||
+      (D->d_cq && !aligned16(w->w_dq)) || !aligned16(q_lat) || !aligned16(q_rope) ||
+      (D->d_cq && D->latent_norm && !aligned16(w->g_q)) || (q_c_out && !aligned16(q_c_out)))
+    return MLA_ERR_INVALID_ARG;
+  Carver cv = carve(ws, ws_bytes);
+  QueryWs q;
+  if (!carve_queries(cv, D, T, !q_c_out, false, &q) || !ws) return MLA_ERR_CAPACITY;
+  __nv_bfloat16* qc = q_c_out ? (__nv_bfloat16*)q_c_out : q.qc;
+  mla_status_t s;
+  if (D->d_cq) {  // c^Q = W^DQ h   (eq 12)
+    GemmCall c{};
+    c.a0 = w->w_dq;
+    c.rows0 = D->d_cq;
+    c.a_row_elems = D->d;
+    c.x = h;
+    c.x_rows = T;
+    c.x_row_elems = D->d;
+    c.K = D->d;
+    c.T = T;
+    c.Z = 1;
+    GemmEpi e{};
+    e.kind = q.cq32 ? EPI_F32 : EPI_BF16;  // fp32 c^Q: the latent RMSNorm writes the bf16 c^Q
+    e.out = q.cq32 ? (void*)q.cq32 : (void*)q.cq;
+    e.out_t = D->d_cq;
+    if ((s = run_gemm(c, e, plan_q1(D, T), st)) != MLA_OK) return s;
+    if (q.cq32 && (s = cq_norm_pass(D, w, q.cq32, q.cq, T, st)) != MLA_OK) return s;
+  }
+  return queries_from_cq(D, w, D->d_cq ? (const void*)q.cq : h, pos, T, qc, q_lat, q_rope, st);
+}
+
+// mla_compress_append followed by mla_absorb_q on the same tokens, with
+// W^DQ sharing the first GEMM with [W^DKV ; W^KR] (all three multiply h):
+// one launch of 5 + 12 row tiles at V2 shapes instead of two.
+static mla_status_t tc_compress_absorb(const mla_layer_desc* D, const mla_weights* w, const void* h,
+                                       const int32_t* seq_idx, const int32_t* pos, int T, mla_paged_cache* cache,
+                                       void* q_lat, void* q_rope, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!D->d_cq) {
+    mla_status_t s = tc_compress_append(D, w, h, seq_idx, pos, T, cache, ws, ws_bytes, st);
+    return s != MLA_OK ? s : tc_absorb_q(D, w, h, pos, T, q_lat, q_rope, ws, ws_bytes, st);
+  }
+  if (!aligned16(h) || !aligned16(w->w_dkv) || !aligned16(w->w_kr) || !aligned16(w->w_dq) ||
+      !aligned16(cache->pool) || !aligned16(w->w_uq) || !aligned16(w->w_qr) || !aligned16(w->w_uk) ||
+      !aligned16(q_lat) || !aligned16(q_rope) || (D->latent_norm && (!aligned16(w->g_kv) || !aligned16(w->g_q))))
+    return MLA_ERR_INVALID_ARG;
+  Carver cv = carve(ws, ws_bytes);
+  QueryWs q;
+  if (!carve_queries(cv, D, T, true, true, &q) || !ws) return MLA_ERR_CAPACITY;
+  // [c^KV ; k^R ; c^Q] = [W^DKV ; W^KR ; W^DQ] h  (eqs 9, 12 + decoupled key)
+  GemmCall c{};
+  c.a0 = w->w_dkv;
+  c.rows0 = D->d_c;
+  c.a1 = w->w_kr;
+  c.rows1 = D->d_hr;
+  c.a2 = w->w_dq;
+  c.rows2 = D->d_cq;
+  c.a_row_elems = D->d;
+  c.x = h;
+  c.x_rows = T;
+  c.x_row_elems = D->d;
+  c.K = D->d;
+  c.T = T;
+  c.Z = 1;
+  GemmEpi e = cache_epi(D, seq_idx, pos, cache, q.lat);
+  e.cq_out = q.cq32 ? (void*)q.cq32 : (void*)q.cq;
+  e.cq_f32 = q.cq32 ? 1 : 0;
+  e.d_cq = D->d_cq;
+  mla_status_t s = run_gemm(c, e, plan_compress_q(D, T), st);
+  if (s != MLA_OK) return s;
+  if (q.lat && (s = kv_second_pass(D, w, q.lat, seq_idx, pos, T, cache, st)) != MLA_OK) return s;
+  if (q.cq32 && (s = cq_norm_pass(D, w, q.cq32, q.cq, T, st)) != MLA_OK) return s;
+  return queries_from_cq(D, w, q.cq, pos, T, q.qc, q_lat, q_rope, st);
 }
 
 // from_o: the input is o [T, n_h, d_h] itself (un-absorbed prefill): W^O only.

@@ -135,10 +135,14 @@ class MLALayer:
     def out_proj(self, st: DecodeState, stream=None):
         mla.out_proj(self.desc, self.cw, st.o_lat, st.u, st.ws, stream)
 
+    def compress_append_absorb_q(self, st: DecodeState, stream=None):
+        mla.compress_append_absorb_q(self.desc, self.cw, st.h, st.seq_idx, st.pos, self.cache(st), st.q_lat,
+                                     st.q_rope, st.ws, stream)
+
     def step(self, st: DecodeState, num_splits: int = 0, stream=None) -> torch.Tensor:
-        """One whole layer step: append, queries, attention, output projection."""
-        self.compress_append(st, stream)
-        self.absorb_q(st, stream)
+        """One whole layer step: append and queries (one call), attention,
+        output projection."""
+        self.compress_append_absorb_q(st, stream)
         self.attend(st, num_splits, stream)
         self.out_proj(st, stream)
         return st.u

@@ -93,6 +93,10 @@ _SIGS = {
     "mla_out_proj_unabsorbed": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "mla_cache_row_bytes": (ctypes.c_size_t, [ctypes.POINTER(LayerDesc)]),
+    "mla_compress_append_absorb_q": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights),
+                                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                                    ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "mla_cache_quantize": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.c_void_p, ctypes.c_longlong,
                                           ctypes.c_void_p, ctypes.c_void_p]),
 }
@@ -179,6 +183,13 @@ def compress_append(desc, w: Weights, h, seq_idx, pos, cache: PagedCache, ws, st
     _check("mla_compress_append", lib().mla_compress_append(
         ctypes.byref(desc), ctypes.byref(w), _ptr(h), _ptr(seq_idx), _ptr(pos), h.shape[0], ctypes.byref(cache),
         _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0, _stream(stream)))
+
+
+def compress_append_absorb_q(desc, w: Weights, h, seq_idx, pos, cache: PagedCache, q_lat, q_rope, ws, stream=None):
+    _check("mla_compress_append_absorb_q", lib().mla_compress_append_absorb_q(
+        ctypes.byref(desc), ctypes.byref(w), _ptr(h), _ptr(seq_idx), _ptr(pos), h.shape[0], ctypes.byref(cache),
+        _ptr(q_lat), _ptr(q_rope), _ptr(ws), ws.numel() * ws.element_size() if ws is not None else 0,
+        _stream(stream)))
 
 
 def absorb_q(desc, w: Weights, h, pos, q_lat, q_rope, ws, stream=None):

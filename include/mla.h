@@ -178,6 +178,15 @@ mla_status_t mla_absorb_q(const mla_layer_desc* desc, const mla_weights* w,
                           const void* h, const int32_t* pos, int T,
                           void* q_lat, void* q_rope, void* ws, size_t ws_bytes, void* stream);
 
+/* mla_compress_append then mla_absorb_q of the same T tokens in one call (same
+ * arguments, results and scratch bound as the two calls).  With query
+ * compression (d_cq > 0) the projections of h by W^DKV, W^KR and W^DQ share
+ * one GEMM launch, so the weights of both steps stream in a single pass. */
+mla_status_t mla_compress_append_absorb_q(const mla_layer_desc* desc, const mla_weights* w, const void* h,
+                                          const int32_t* seq_idx, const int32_t* pos, int T,
+                                          mla_paged_cache* cache, void* q_lat, void* q_rope, void* ws,
+                                          size_t ws_bytes, void* stream);
+
 /* Decode attention over the latent cache, one query per sequence.
  *   q_lat [B, n_h, d_c], q_rope [B, n_h, d_hr]
  *   kv_len [B] int32     rows attended by sequence b (including the token just

@@ -470,3 +470,22 @@ def test_fp8_prefill_chunk():
             r = b * 9 + q
             assert_bf16(np32(st.o_lat)[r], outs[q]["o_lat"], f"o_lat {b},{q}")
             assert_bf16(np32(st.u)[r], outs[q]["u"], f"u {b},{q}")
+
+
+@pytest.mark.parametrize("w", [V2_SMALL, _with_norm(V2_SMALL, "v2_norm_fused"), LITE_SMALL], ids=lambda w: w.name)
+def test_fused_append_and_queries_equal_the_two_calls(w):
+    # mla_compress_append_absorb_q shares one GEMM between [W^DKV; W^KR] and
+    # W^DQ; each tile's K split and reduction order are those of the separate
+    # launches, so cache rows and queries are bit-identical
+    batch = I.gen_batch(w)
+    layer = MLALayer(w.dims, weights_for(w))
+    a, b = layer.upload(batch), layer.upload(batch)
+    layer.compress_append(a)
+    layer.absorb_q(a)
+    layer.compress_append_absorb_q(b)
+    torch.cuda.synchronize()
+    assert mla.get_last_error() == 0
+    # bit patterns: unwritten slots hold NaN, which never equals itself
+    assert torch.equal(a.pool.view(torch.int16), b.pool.view(torch.int16))
+    assert torch.equal(a.q_lat.view(torch.int16), b.q_lat.view(torch.int16))
+    assert torch.equal(a.q_rope.view(torch.int16), b.q_rope.view(torch.int16))
