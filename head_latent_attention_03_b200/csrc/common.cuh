@@ -250,6 +250,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// The same with f16 A and B (kind::f16 takes either type; A and B match).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)  // D format: f32; A, B format: f16 (0)
+         | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
 // UMMA shared-memory descriptor (sm_100 version 1).
 // layout: 0 none, 2 = 128B swizzle, 4 = 64B, 6 = 32B.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
@@ -498,17 +505,25 @@ __device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
   return r;
 }
 
-// Two E4M3 codes (low byte = element 0) times 2^e as two bf16 (element 0 in
-// the low half), exactly: the codes become f16 (every E4M3 value is a normal
-// f16 except 0), and the f16 exponent field is rebased to bf16's bias plus e
-// (bias_e = (112 + e) << 7; the f16 mantissa's three used bits shift into
-// bf16's top mantissa bits).  Zeros stay zero.  Exact for e >= -112.
-__device__ __forceinline__ uint32_t bf16x2_from_e4m3x2(uint16_t codes, uint32_t bias_e) {
-  uint32_t h;
+// Two E4M3 codes (low byte = element 0) times sc2 (a power of two in both
+// f16 halves) as two f16, element 0 in the low half: the codes convert to f16
+// exactly and the product is exact while it stays in f16's normal range.
+__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint16_t codes, uint32_t sc2) {
+  uint32_t h, r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(codes));
-  const uint32_t mag = h & 0x7FFF7FFFu;
-  const uint32_t nz = ((mag + 0x7FFF7FFFu) >> 15) & 0x00010001u;  // 1 in each non-zero half
-  return ((mag >> 3) + nz * bias_e) | (h & 0x80008000u);
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(sc2));
+  return r;
+}
+// Two bf16 (element 0 in the low half) as two f16, rounded to nearest even.
+__device__ __forceinline__ uint32_t f16x2_from_bf16x2(uint32_t w) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(__uint_as_float(w & 0xFFFF0000u)), "f"(__uint_as_float(w << 16)));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Byte offset inside a swizzled (SW32/64/128) region: the 16-byte chunk index

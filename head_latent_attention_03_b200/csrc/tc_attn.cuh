@@ -65,7 +65,7 @@ struct AttnCfg {
   static constexpr int CONV = F8 ? NL : 0;             // F8: "slot converted" barriers
   static constexpr int OFF_SCALE = OFF_LAT + NL * LAT_SLOT;
   static constexpr int OFF_BAR = OFF_SCALE + NSC * SC_SLOT;
-  static constexpr int N_BAR = 2 * NL + 2 * NR + 1 + 2 + 2 + 2 + 2 + 1 + CONV + 2 * NSC;
+  static constexpr int N_BAR = 2 * NL + 2 * NR + 1 + 2 + 2 + 2 + 2 + 1 + CONV + 2 * NSC + (F8 ? 1 : 0);
   static constexpr int OFF_RED = OFF_BAR + N_BAR * 8 + 16;
   static constexpr int SMEM = OFF_RED + 2 * 4 * H * 4 + 1024;
   static constexpr int TMEM_COLS = 6 * H <= 128 ? 128 : 256;
@@ -349,7 +349,8 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
   uint64_t* lat_conv = grp_bar + 1;  // F8: latent slot converted to bf16 (128 converter arrivals)
   uint64_t* sc_full = lat_conv + C::CONV;
   uint64_t* sc_empty = sc_full + C::NSC;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sc_empty + C::NSC);
+  uint64_t* q_conv = sc_empty + C::NSC;  // F8: the segment's queries converted to f16 (128 arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_conv + (F8 ? 1 : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [2][4][H]
 
@@ -382,6 +383,7 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
       mbar_init(&sc_full[i], 1);
       mbar_init(&sc_empty[i], 128);
     }
+    if (F8) mbar_init(q_conv, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -491,8 +493,10 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
     // written.  PV(j) frees the slots that QK(j+1) waits for, so neither may
     // block the other.
     if (elect_one()) {
-      const uint32_t id_qk = idesc_bf16_f32(ATT_TILE, H, false, false);
-      const uint32_t id_pv = idesc_bf16_f32(ATT_TILE, H, true, true);
+      // F8: the latent tile, Q's latent chunks and P are f16; the RoPE chunk stays bf16
+      const uint32_t id_qr = idesc_bf16_f32(ATT_TILE, H, false, false);
+      const uint32_t id_qk = F8 ? idesc_f16_f32(ATT_TILE, H, false, false) : id_qr;
+      const uint32_t id_pv = F8 ? idesc_f16_f32(ATT_TILE, H, true, true) : idesc_bf16_f32(ATT_TILE, H, true, true);
       const uint32_t q_base = smem_u32(smem + C::OFF_Q);
       const uint32_t lat_base = smem_u32(smem + C::OFF_LAT);
       const uint32_t rope_base = smem_u32(smem + C::OFF_ROPE);
@@ -532,7 +536,7 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
           const int jq = cq.g;
           const int sb = jq & 1;
           if (!sbuf_ok) sbuf_ok = jq < 2 || mbar_test(smem_u32(&s_free[sb]), ((jq >> 1) - 1) & 1);
-          if (q_seen != cq.n && mbar_test(smem_u32(q_full), cq.n & 1)) q_seen = cq.n;
+          if (q_seen != cq.n && mbar_test(smem_u32(F8 ? q_conv : q_full), cq.n & 1)) q_seen = cq.n;
           if (sbuf_ok && q_seen == cq.n) {
             bool ready;
             uint32_t ka;
@@ -556,7 +560,7 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t ad = smem_desc(ka + kk * 32, 16, 1024, SW128);
                 const uint64_t bd = smem_desc(q_base + qchunk * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
-                mma_bf16_ss(tS + sb * H, ad, bd, id_qk, (kq | kk) != 0 ? 1u : 0u);
+                mma_bf16_ss(tS + sb * H, ad, bd, kq == 0 ? id_qr : id_qk, (kq | kk) != 0 ? 1u : 0u);
               }
               if (kq == 0) mma_commit(&rope_empty[jq % C::NR]);
               if (++kq == 9) {
@@ -589,12 +593,14 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
     }
   } else if (F8 && warp >= 6) {
     // ------------------------------------------------------------ F8 converters
-    // Thread = (page p, token row r) of every latent slot: it reads the
-    // row's 128 codes from the slot's upper half and writes them as bf16
-    // times the row's scale 2^e into both halves in the MMA's SW128 layout
-    // (codes of columns 0..63 -> the lower half, 64..127 -> the upper half,
-    // over exactly the bytes this thread just read, so no other thread's
-    // input is touched).
+    // Per segment: the queries' latent chunks, bf16 -> f16 in place.  Per
+    // tile: thread = (page p, token row r) of every latent slot; it reads the
+    // row's 128 codes from the slot's upper half and writes code * 2^e as f16
+    // into both halves in the MMA's SW128 layout (codes of columns 0..63 ->
+    // the lower half, 64..127 -> the upper half, over exactly the bytes this
+    // thread just read, so no other thread's input is touched).  The f16
+    // values are exact for scales 2^e with -15 <= e <= 7 (latent values of
+    // magnitude 2^-6 .. 2^15 at the row maximum).
     const int ct = threadIdx.x - ATT_THREADS;
     const int p = ct >> 6, r = ct & 63;
     TileCursor c;
@@ -602,14 +608,24 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
     bool ok = true;
     while (ok && !c.done()) {
       const int g = c.g;
+      if (c.first()) {
+        if (!mbar_wait(q_full, c.n & 1, abort_flag, 433)) break;
+        uint4* q = reinterpret_cast<uint4*>(smem + C::OFF_Q);
+        for (int i = ct; i < 8 * C::Q_CHUNK / 16; i += 128) {
+          const uint4 w = q[i];
+          q[i] = make_uint4(f16x2_from_bf16x2(w.x), f16x2_from_bf16x2(w.y), f16x2_from_bf16x2(w.z),
+                            f16x2_from_bf16x2(w.w));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(q_conv);
+      }
       const int ss = g % 2;
       if (!mbar_wait(&sc_full[ss], (g / 2) & 1, abort_flag, 431)) break;
       const float scale = *reinterpret_cast<const float*>(smem + C::OFF_SCALE + ss * C::SC_SLOT + p * 1024 + r * 16);
       mbar_arrive(&sc_empty[ss]);
-      // bf16 exponent rebase plus e for both halves (a zero-filled row past
-      // the cache has scale 0: any value, its codes are all zero)
-      const int e = (int)((__float_as_uint(scale) >> 23) & 0xFFu) - 127;
-      const uint32_t bias = ((uint32_t)(112 + e) & 0xFFu) << 7;
+      // 2^e in both f16 halves (a zero-filled row past the cache has scale 0:
+      // its codes are zero as well)
+      const uint32_t sc2 = pack_f16(scale, scale);
       for (int m = 0; m < 4 && ok; ++m) {
         const int li = 4 * g + m, s = li % C::NL;
         if (!mbar_wait(&lat_full[s], (li / C::NL) & 1, abort_flag, 432)) {
@@ -625,18 +641,18 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
         for (int j = 0; j < 8; ++j) v[j] = in[(j + r) & 7];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          // codes 16k .. 16k+15: bf16 columns 16(k%4) .. +15 of half k/4, 16-byte units 2(k%4), 2(k%4)+1
+          // codes 16k .. 16k+15: f16 columns 16(k%4) .. +15 of half k/4, 16-byte units 2(k%4), 2(k%4)+1
           const int k = (j + r) & 7;
           uint8_t* half = slot + (k >> 2) * 16384;
           const uint32_t u0 = 2u * (k & 3);
-          const uint4 lo = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[j].x, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[j].x >> 16), bias),
-                                      bf16x2_from_e4m3x2((uint16_t)v[j].y, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[j].y >> 16), bias));
-          const uint4 hi = make_uint4(bf16x2_from_e4m3x2((uint16_t)v[j].z, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[j].z >> 16), bias),
-                                      bf16x2_from_e4m3x2((uint16_t)v[j].w, bias),
-                                      bf16x2_from_e4m3x2((uint16_t)(v[j].w >> 16), bias));
+          const uint4 lo = make_uint4(f16x2_from_e4m3x2((uint16_t)v[j].x, sc2),
+                                      f16x2_from_e4m3x2((uint16_t)(v[j].x >> 16), sc2),
+                                      f16x2_from_e4m3x2((uint16_t)v[j].y, sc2),
+                                      f16x2_from_e4m3x2((uint16_t)(v[j].y >> 16), sc2));
+          const uint4 hi = make_uint4(f16x2_from_e4m3x2((uint16_t)v[j].z, sc2),
+                                      f16x2_from_e4m3x2((uint16_t)(v[j].z >> 16), sc2),
+                                      f16x2_from_e4m3x2((uint16_t)v[j].w, sc2),
+                                      f16x2_from_e4m3x2((uint16_t)(v[j].w >> 16), sc2));
           *reinterpret_cast<uint4*>(half + ((u0 ^ (uint32_t)(r & 7)) << 4)) = lo;
           *reinterpret_cast<uint4*>(half + (((u0 + 1) ^ (uint32_t)(r & 7)) << 4)) = hi;
         }
@@ -744,7 +760,7 @@ __global__ void __launch_bounds__(AttnCfg<H, F8>::THREADS, 1)
         const float p1 = valid ? exp2_approx(s[h + 1] - m_run[h + 1]) : 0.f;
         l_part[h] += p0;
         l_part[h + 1] += p1;
-        pk[h / 2] = pack_bf16(p0, p1);
+        pk[h / 2] = F8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
       }
       // the P buffer was last read by PV(j-2)
       if (j >= 2 && !mbar_wait(&pv_done[sb], ((j - 2) >> 1) & 1, abort_flag, 423)) {
