@@ -283,7 +283,7 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
         after = lambda: mla.out_proj_unabsorbed(layer.desc, layer.cw, st.o, st.u)
     else:
         attn_bytes, attn_flops = workload_work(w, batch)
-        calls = [lambda: layer.compress_append(st), lambda: layer.absorb_q(st)]
+        calls = [lambda: layer.compress_append_absorb_q(st)]
         attend = lambda: layer.attend(st)
         after = lambda: layer.out_proj(st)
     stream = torch.cuda.current_stream()
@@ -390,8 +390,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     def step(ev_pair=None):
-        layer.compress_append(st)
-        layer.absorb_q(st)
+        layer.compress_append_absorb_q(st)
         if ev_pair is not None:
             ev_pair[0].record(stream)
         layer.attend(st)
@@ -413,7 +412,10 @@ def run_ours(args):
         t_pre = time.time()
         while time.time() - t_pre < 0.6:
             step()
-    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    def pairs(n):
+        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+
+    # (1) the headline: K whole steps back to back, nothing between the kernels
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -421,12 +423,26 @@ def run_ours(args):
     n0 = mla.launch_count()
     e0.record(stream)
     for k in range(args.steps):
-        step(attn_ev[k])
+        step()
     e1.record(stream)
     torch.cuda.synchronize()
     n_launch = mla.launch_count() - n0
     if world > 1:
         dist.barrier()
+    # (2) the attention stage (plan + attention kernel + combine) of each step,
+    # between events, and (3) the attention kernel alone, between events the
+    # library records around it (mla_debug_attention_events)
+    attn_ev, kern_ev = pairs(args.steps), pairs(args.steps)
+    for a, b in kern_ev:  # create the events
+        a.record(stream)
+        b.record(stream)
+    for k in range(args.steps):
+        step(attn_ev[k])
+    for k in range(args.steps):
+        mla.debug_attention_events(*kern_ev[k])
+        step()
+    mla.debug_attention_events(None, None)
+    torch.cuda.synchronize()
     clocks = sampler.stop() if not args.profile_run else {"sm_mhz": None, "sm_max_mhz": None,
                                                           "reasons": ["not sampled (profile run)"]}
     code = mla.get_last_error()
@@ -434,7 +450,8 @@ def run_ours(args):
         raise RuntimeError(f"device status after timed steps: {mla.status_string(code)}")
     t_ms = e0.elapsed_time(e1)
     attn_ms = sum(a.elapsed_time(b) for a, b in attn_ev) / args.steps
-    t_ms, attn_ms = max_over_ranks([t_ms, attn_ms], dev)
+    kern_ms = sum(a.elapsed_time(b) for a, b in kern_ev) / args.steps
+    t_ms, attn_ms, kern_ms = max_over_ranks([t_ms, attn_ms, kern_ms], dev)
 
     # end to end through the public API: pinned host inputs in, result out, every step
     h_host = st.h.cpu().pin_memory()
@@ -486,6 +503,11 @@ def run_ours(args):
         roof.update({"traffic": traffic,
                      "kernel": f"attention stage timed as one: mla_attn_plan_kernel + {attn_kernel} + mla_combine_kernel"
                                f" (traffic: {attn_kernel} alone)"})
+        k_roof = roofline_of(attn_bytes, attn_flops, kern_ms, peaks, peak_src)
+        roof["kernel_only"] = {"kernel": attn_kernel, "us": round(kern_ms * 1e3, 2), "bound": k_roof["bound"],
+                               "achieved": k_roof["achieved"], "unit": k_roof["unit"], "frac": k_roof["frac"],
+                               "timed": "CUDA events the library records on the launch stream right before and "
+                                        "after the attention kernel, in separate steps"}
         value = world * rows * args.steps / (t_ms * 1e-3)
         e2e_value = world * rows * e2e_steps / (t_e2e * 1e-3) if e2e_steps else None
         out = {

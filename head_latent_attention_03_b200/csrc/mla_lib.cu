@@ -398,6 +398,11 @@ int mla_trace_read(void* dst, size_t bytes) {
 }
 #endif
 
+void mla_debug_attention_events(void* before, void* after) {
+  g_attn_ev_before = reinterpret_cast<cudaEvent_t>(before);
+  g_attn_ev_after = reinterpret_cast<cudaEvent_t>(after);
+}
+
 mla_status_t mla_get_last_error(void* stream) {
   if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return MLA_ERR_CUDA;
   int code = 0, zero = 0;

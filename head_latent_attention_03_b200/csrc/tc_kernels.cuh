@@ -931,6 +931,11 @@ static cudaError_t launch_attn(const CUtensorMap& mq, const CUtensorMap& mr, con
   return launch_pdl(kfn, grid, dim3(AttnCfg<H, false>::THREADS), smem, st, 1, mq, mr, mc, mc, mc, a);
 }
 
+// Measurement hook (mla_debug_attention_events): events recorded on the
+// attention call's stream right before and after its attention kernel (after
+// the work plan, before the combine), so that the kernel alone can be timed.
+inline cudaEvent_t g_attn_ev_before = nullptr, g_attn_ev_after = nullptr;
+
 // kv_begin (partial decode): rows [kv_begin[b], kv_len[b]) only, every row
 // written in fp32 to o_f32 (o_lat unused) with its lse.
 static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, const void* q_rope,
@@ -991,6 +996,7 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   a.o_part = aw.o_part;
   a.lse_part = aw.lse_part;
   cudaError_t e;
+  if (g_attn_ev_before && cudaEventRecord(g_attn_ev_before, st) != cudaSuccess) return MLA_ERR_CUDA;
   if (pair) {
     CUtensorMap m1, m2;
     if (!map_cache_chunks(&m1, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 1) ||
@@ -1006,6 +1012,7 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
                 : launch_attn<32>(mq, mr, mc, mr8, ms8, f8, a, grid, st);
   }
   if (e != cudaSuccess) return MLA_ERR_CUDA;
+  if (g_attn_ev_after && cudaEventRecord(g_attn_ev_after, st) != cudaSuccess) return MLA_ERR_CUDA;
   if (p.max_slots > 0) {
     // enough blocks for two per SM: split the latent columns when there are few rows
     const int blocks = rows * (D->n_h / COMBINE_HEADS);

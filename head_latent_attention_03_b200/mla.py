@@ -93,6 +93,7 @@ _SIGS = {
     "mla_out_proj_unabsorbed": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights), ctypes.c_void_p,
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "mla_cache_row_bytes": (ctypes.c_size_t, [ctypes.POINTER(LayerDesc)]),
+    "mla_debug_attention_events": (None, [ctypes.c_void_p, ctypes.c_void_p]),
     "mla_compress_append_absorb_q": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights),
                                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                                     ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_void_p,
@@ -162,6 +163,14 @@ def launch_count() -> int:
 
 def status_string(code: int) -> str:
     return lib().mla_status_string(code).decode()
+
+
+def debug_attention_events(before=None, after=None):
+    """Record torch.cuda.Event `before` / `after` around every attention kernel
+    from now on (None, None: stop).  The events must have been recorded once
+    (so that they exist)."""
+    lib().mla_debug_attention_events(before.cuda_event if before is not None else None,
+                                     after.cuda_event if after is not None else None)
 
 
 def cache_row_bytes(desc: LayerDesc) -> int:

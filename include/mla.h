@@ -311,6 +311,16 @@ mla_status_t mla_out_proj(const mla_layer_desc* desc, const mla_weights* w, cons
  * abandoned wait) or MLA_ERR_CUDA if the stream reported a CUDA error. */
 mla_status_t mla_get_last_error(void* stream);
 
+/* Measurement hook.  With non-NULL handles (cudaEvent_t values), every
+ * later bf16 attention call (decode, no-alloc, partial, latent prefill)
+ * records `before` on its stream right before its attention kernel (after
+ * the work plan) and `after` right after it (before the combine), so that
+ * the kernel can be timed alone; the events separate the kernel from its
+ * neighbours on the stream, so a timed run with them set is not the
+ * pipelined step.  NULL, NULL turns it off.  Process-wide, not thread-safe:
+ * for benchmarks only. */
+void mla_debug_attention_events(void* before, void* after);
+
 /* Static string for a status code. */
 const char* mla_status_string(mla_status_t status);
 
