@@ -323,6 +323,21 @@ def test_gather_rows_returns_rows_in_token_order():
         assert np.array_equal(got, want.astype(np.float64)), b
 
 
+def test_gather_rows_hand_computed_lookup():
+    # a fixed 3-page pool of 4-slot pages whose row values encode (page,
+    # slot); the table sends token j of the sequence to page [2, 0, 1][j // 4],
+    # slot j % 4.  Token 5 sits on page 0 slot 1, token 9 on page 1 slot 1,
+    # token 2 on page 2 slot 2 (worked out by hand from that table).
+    pool = np.array([[[10 * p + s, -(10 * p + s)] for s in range(4)] for p in range(3)], dtype=np.float64)
+    table = np.array([2, 0, 1], dtype=np.int32)
+    rows = O.gather_rows(pool, table, 10, 4)
+    assert rows.shape == (10, 2)
+    assert rows[5].tolist() == [1.0, -1.0]
+    assert rows[9].tolist() == [11.0, -11.0]
+    assert rows[2].tolist() == [22.0, -22.0]
+    assert rows[0].tolist() == [20.0, -20.0] and rows[4].tolist() == [0.0, 0.0]
+
+
 # Data flow of the decoupled RoPE parts ([explainer] 2.2.2): the shared key
 # k^R is computed from h_t itself, not from the latent c^KV, and both query
 # parts come from the query latent c^Q.  Zeroing W^DKV must leave k^R intact;
