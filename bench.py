@@ -2,7 +2,7 @@
 """Benchmark of the MLA decode layer step on B200 (one JSON line on stdout).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload v2|lite|lite_fp8|long|prefill] [--no-cpu-baseline] [--no-extra]
+                    [--workload v2|v2_fp8|lite|lite_fp8|long|prefill] [--no-cpu-baseline] [--no-extra]
 
 A step is one pass of the whole hot path over one batch: compress_append ->
 absorb_q -> decode attention (+ LSE combine) -> out_proj, through the C ABI.
@@ -43,6 +43,8 @@ WORKLOAD_TEXT = {
           "decode batch 64, prior cache lengths uniform in [1,8192], block 64, permuted page table",
     "lite": "DeepSeek-V2-Lite-shaped MLA layer (d=2048, n_h=16, d_h=128, d_c=512, d_h^R=64), bf16, "
             "decode batch 32, 4096 prior tokens each, block 64",
+    "v2_fp8": "the V2 workload over an FP8 latent cache (E4M3 codes of c^KV with a power-of-two scale per row, "
+              "bf16 k^R: 656 bytes per token), bf16 compute",
     "lite_fp8": "the V2-Lite workload over an FP8 latent cache (E4M3 codes of c^KV with a power-of-two scale "
                 "per row, bf16 k^R: 656 bytes per token), bf16 compute",
     "long": "V2-shaped MLA layer, bf16, decode batch 4 over 131072 prior tokens each, YaRN s=40, split-KV",
@@ -343,7 +345,7 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
 
 
 # Steps of the extra workloads (their steps are longer than the headline's).
-EXTRA_STEPS = {"lite": (100, 5), "lite_fp8": (100, 5), "long": (20, 3), "prefill": (2, 1)}
+EXTRA_STEPS = {"lite": (100, 5), "lite_fp8": (100, 5), "v2_fp8": (100, 5), "long": (20, 3), "prefill": (2, 1)}
 
 
 # ---------------------------------------------------------------------------
@@ -491,7 +493,7 @@ def run_ours(args):
     if not args.no_extra and not args.profile_run:
         del layer, st
         torch.cuda.empty_cache()
-        for name in ("lite", "lite_fp8", "long", "prefill"):
+        for name in ("lite", "lite_fp8", "v2_fp8", "long", "prefill"):
             if name != args.workload:
                 k, wu = EXTRA_STEPS[name]
                 extra[name] = measure_extra(name, k, wu, dev, peaks, peak_src)
@@ -499,7 +501,8 @@ def run_ours(args):
     if rank == 0:
         roof = roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src)
         traffic = committed_traffic(args.workload)
-        attn_kernel = "mla_attn_pair_kernel" if w.dims.n_h == 128 else "mla_attn_kernel"
+        attn_kernel = ("mla_attn_pair_kernel" if w.dims.n_h == 128 and getattr(w.dims, "cache_dtype", "bf16") != "fp8"
+                       else "mla_attn_kernel")
         roof.update({"traffic": traffic,
                      "kernel": f"attention stage timed as one: mla_attn_plan_kernel + {attn_kernel} + mla_combine_kernel"
                                f" (traffic: {attn_kernel} alone)"})
@@ -595,7 +598,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=["v2", "lite", "lite_fp8", "long", "prefill"], default="v2")
+    ap.add_argument("--workload", choices=["v2", "v2_fp8", "lite", "lite_fp8", "long", "prefill"], default="v2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--profile-run", action="store_true",

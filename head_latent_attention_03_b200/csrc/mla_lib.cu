@@ -40,9 +40,9 @@ bool desc_valid(const mla_layer_desc* D) {
   return D->dtype == MLA_F32 || D->dtype == MLA_BF16;
 }
 
-// The latent attention kernels that read FP8 rows: the one-CTA kernel
-// (n_h <= 64); the CTA-pair kernel (n_h = 128) reads bf16 rows only.
-bool attn_cache_supported(const mla_layer_desc* D) { return !fp8_cache(D) || !use_pair_kernel(D); }
+// Every latent attention path reads both row formats (FP8 rows of a 128-head
+// layer go to the one-CTA kernel, see use_pair_kernel).
+bool attn_cache_supported(const mla_layer_desc*) { return true; }
 
 // Shapes the tcgen05 kernels are written for.
 bool bf16_supported(const mla_layer_desc* D) {

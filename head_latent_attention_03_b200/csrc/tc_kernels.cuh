@@ -35,6 +35,9 @@ inline int num_sms() {
   return n > 0 ? n : 148;
 }
 
+// the layer's cache rows are FP8 (E4M3 codes of c^KV, bf16 k^R, a scale)
+inline bool fp8_cache(const mla_layer_desc* D) { return D->cache_dtype == MLA_CACHE_FP8_E4M3; }
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -368,7 +371,6 @@ inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
 
 // Workspace of the projections: only the bf16 intermediates between two
 // GEMMs (K splits are reduced inside each GEMM's cluster).
-inline bool fp8_cache(const mla_layer_desc* D) { return D->cache_dtype == MLA_CACHE_FP8_E4M3; }
 // bytes of one cache row: [c^KV | k^R] in bf16, or the FP8 row (codes, bf16
 // k^R, scale, padding)
 inline int cache_row_bytes(const mla_layer_desc* D) {
@@ -399,8 +401,11 @@ inline size_t ws_out(const mla_layer_desc* D, int T) {
 }
 
 inline int heads_per_cta(const mla_layer_desc* D) { return D->n_h == 16 ? 16 : 32; }
-// 128-head layers run on CTA pairs (tc_attn2.cuh), one pair per (row, split)
-inline bool use_pair_kernel(const mla_layer_desc* D) { return D->n_h == 128; }
+// 128-head layers with bf16 rows run on CTA pairs (tc_attn2.cuh), one pair
+// per (row, split); over FP8 rows they run on the one-CTA kernel as four
+// 32-head groups per worker, side by side on the same tiles (L2 serves the
+// other three groups).
+inline bool use_pair_kernel(const mla_layer_desc* D) { return D->n_h == 128 && !fp8_cache(D); }
 
 // Host side of the attention work plan (the device side is
 // mla_attn_plan_kernel).  Automatic decode plans deal the tiles of all rows

@@ -92,8 +92,10 @@ WORKLOADS: Dict[str, Workload] = {
     "v2": Workload("v2", 3, V2, 64, "uniform:1:8192", permute_pages=True),
     "long": Workload("long", 4, V2_YARN, 4, "fixed:131072"),
     "prefill": Workload("prefill", 5, V2, 8, "fixed:4096", new_tokens=4096),
-    # the V2-Lite workload (same draws) over an FP8 latent cache
+    # the V2-Lite and V2 workloads (same draws) over an FP8 latent cache
     "lite_fp8": Workload("lite_fp8", 2, dataclasses.replace(LITE, cache_dtype="fp8"), 32, "fixed:4096"),
+    "v2_fp8": Workload("v2_fp8", 3, dataclasses.replace(V2, cache_dtype="fp8"), 64, "uniform:1:8192",
+                       permute_pages=True),
 }
 
 # tensor ids inside a workload's seed tree

@@ -67,12 +67,13 @@ def test_fp8_cache_rows_and_limits_without_a_gpu(lib):
     assert mla.cache_row_bytes(fp8) == 656
     # FP8 rows need a bf16 layer: an fp32 layer with them is an invalid desc
     assert mla.cache_row_bytes(mla.layer_desc(dataclasses.replace(TINY, cache_dtype="fp8"))) == 0
-    # the 128-head CTA-pair attention reads bf16 rows only: refused on the
+    # the un-absorbed prefill decompresses bf16 rows only: refused on the
     # host, before any CUDA call (the pointers are never dereferenced)
     v2 = mla.layer_desc(dataclasses.replace(V2, cache_dtype="fp8"))
     cache = mla.PagedCache(16, 1, 16, 1)
-    code = mla.lib().mla_decode_attn(ctypes.byref(v2), 16, 16, ctypes.byref(cache), 16, 1, 16, 1 << 20, 0, 16,
-                                     None, None)
+    w = mla.Weights(*([16] * 10))
+    code = mla.lib().mla_prefill_attn_unabsorbed(ctypes.byref(v2), ctypes.byref(w), 16, 16, ctypes.byref(cache),
+                                                 16, 4, 1, 16, 1 << 20, 16, None, None)
     assert code == 2
     # encoding rows into the FP8 format needs a desc with FP8 rows
     assert mla.lib().mla_cache_quantize(ctypes.byref(mla.layer_desc(LITE)), 16, 1, 32, None) == 1

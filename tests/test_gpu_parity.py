@@ -445,6 +445,19 @@ def test_fp8_decode_with_latent_norm():
     check_decode(w)
 
 
+def test_fp8_decode_v2_small():
+    # 128 heads over FP8 rows: the one-CTA kernel as four 32-head groups
+    w = dataclasses.replace(I.WORKLOADS["v2_fp8"], name="v2_fp8_small", batch=3, prior="list:127,128,1000")
+    check_decode(w)
+
+
+def test_fp8_v2_full_size_sampled():
+    # the V2 workload over an FP8 cache: two sequences through the oracle
+    w = I.WORKLOADS["v2_fp8"]
+    lens = I.prior_lengths(w)
+    check_decode(w, seqs=[int(np.argmin(lens)), int(np.argmax(lens))])
+
+
 def test_fp8_full_size_sampled():
     # 32 x 4096 prior tokens (the V2-Lite workload over an FP8 cache): two
     # sequences through the oracle
