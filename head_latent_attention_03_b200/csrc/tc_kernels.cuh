@@ -22,6 +22,7 @@
 #include "tc_attn2.cuh"
 #include "tc_gemm.cuh"
 #include "tc_prefill.cuh"
+#include "tc_gemm_heads.cuh"
 
 namespace mla {
 
@@ -361,9 +362,6 @@ inline GemmPlan plan_q2(const mla_layer_desc* D, int T) {
   const int q_in = D->d_cq ? D->d_cq : D->d;
   return plan_gemm((D->n_h * D->d_h + 127) / 128 + (D->n_h * D->d_hr + 127) / 128, 1, T, q_in);
 }
-inline GemmPlan plan_q3(const mla_layer_desc* D, int T) {
-  return plan_gemm(D->d_c / 128, D->n_h, T, D->d_h, /*a_mn=*/true);
-}
 inline GemmPlan plan_o1(const mla_layer_desc* D, int T) { return plan_gemm((D->d_h + 127) / 128, D->n_h, T, D->d_c); }
 inline GemmPlan plan_o2(const mla_layer_desc* D, int T) {
   return plan_gemm((D->d + 127) / 128, 1, T, D->n_h * D->d_h);
@@ -649,29 +647,28 @@ static mla_status_t queries_from_cq(const mla_layer_desc* D, const mla_weights* 
     if ((s = run_gemm(c, e, plan_q2(D, T), st)) != MLA_OK) return s;
   }
   if (!q_lat) return MLA_OK;  // queries only (the un-absorbed prefill reads q^C)
-  {  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major
-    GemmCall c{};
-    c.a0 = w->w_uk;
-    c.rows0 = D->d_c;
-    c.a_row_elems = D->d_c;
-    c.a_mn = true;
-    c.a_mn_rows = D->n_h * D->d_h;
-    c.x = qc;
-    c.x_rows = T;
-    c.x_row_elems = nq;
-    c.K = D->d_h;
-    c.T = T;
-    c.Z = D->n_h;
-    c.a_z_rows = D->d_h;
-    c.b_z_cols = D->d_h;
-    GemmEpi e{};  // q_lat[t][head][c]
-    e.kind = EPI_BF16;
-    e.out = q_lat;
-    e.out_z = D->d_c;
-    e.out_t = (long long)D->n_h * D->d_c;
-    if ((s = run_gemm(c, e, plan_q3(D, T), st)) != MLA_OK) return s;
-  }
-  return MLA_OK;
+  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major, all
+  // (head, row tile, token tile) units on one persistent CTA per SM
+  CUtensorMap mA, mB;
+  if (!map_2d(&mA, w->w_uk, (uint64_t)D->d_c, (uint64_t)D->n_h * D->d_h, (uint64_t)D->d_c * 2, 64, 64) ||
+      !map_rows_chunks(&mB, qc, (uint64_t)nq, (uint64_t)T, (uint64_t)nq * 2, (uint32_t)HeadsCfg::TN, 1))
+    return MLA_ERR_CUDA;
+  HeadsArgs ha;
+  ha.n_h = D->n_h;
+  ha.d_h = D->d_h;
+  ha.d_c = D->d_c;
+  ha.T = T;
+  ha.k_chunks = D->d_h / 64;
+  ha.m_tiles = D->d_c / 128;
+  ha.n_tiles = (T + HeadsCfg::TN - 1) / HeadsCfg::TN;
+  ha.units = D->n_h * ha.m_tiles * ha.n_tiles;
+  ha.out = (__nv_bfloat16*)q_lat;
+  cudaFuncSetAttribute(mla_absorb_heads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HeadsCfg::SMEM);
+  const int grid = std::min(ha.units, num_sms());
+  return launch_pdl(mla_absorb_heads_kernel, dim3(grid), dim3(HeadsCfg::THREADS), HeadsCfg::SMEM, st, 1, mA, mB,
+                    ha) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 // q_c_out: write q^C [T, n_h, d_h] there (the un-absorbed prefill's queries);
