@@ -1,27 +1,31 @@
-// tc_gemm_heads.cuh — the per-head absorbed query projection as one
+// tc_gemm_heads.cuh — the per-head projections of the absorbed form as one
 // persistent tcgen05 kernel:
 //
-//   q_lat[t][i][n] = sum_k W^UK[i d_h + k][n] q^C[t][i d_h + k]
-//                                     (q_lat_i = (W^UK_i)^T q^C_i, DeepSeek-V2
-//                                      explainer, adg.csdn.net, section 2.2.2)
+//   q_lat[t][i][n] = sum_k W^UK[i d_h + k][n] q^C[t][i d_h + k]   (A_MN: W^UK read MN-major)
+//   o[t][i][r]     = sum_c W^UV[i d_h + r][c] o_lat[t][i][c]      (W^UV read K-major)
+// (q_lat_i = (W^UK_i)^T q^C_i and o_i = W^UV_i o_lat_i: W^UK absorbed into the
+// query, W^UV applied before W^O — DeepSeek-V2 explainer, adg.csdn.net,
+// section 2.2.2; "DeepSeek-V2" reading notes, eq 11.)
 //
-// Each head contributes d_c / 128 output tiles of 128 latent rows over a
-// short contraction (K = d_h = 128): 512 small tiles at V2 shapes, each a
-// 32 KB slice of W^UK.  Launched one CTA per tile they spend their life in
-// set-up; here 1 CTA per SM walks a contiguous range of (head, row tile,
-// token tile) units, the weight loads stream through one ring of stages
-// across unit boundaries, and the accumulator is double-buffered in TMEM so
-// that a unit's epilogue overlaps the next unit's MMAs.
+// Each head contributes a few output tiles of 128 rows: q_lat has d_c / 128
+// tiles per head over a short contraction (K = d_h = 128, 512 tiles of 32 KB
+// of W^UK at V2 shapes); o has one tile per head over K = d_c.  Launched one
+// CTA per tile they spend their life in set-up; here 1 CTA per SM walks a
+// contiguous range of (head, row tile, token tile) units, the weight loads
+// stream through one ring of stages across unit boundaries, and the
+// accumulator is double-buffered in TMEM so that a unit's epilogue overlaps
+// the next unit's MMAs.
 //
 // Operands: A = W^UK_i read MN-major (two 64-column SW128 boxes per 64-row K
-// chunk: the head's [d_h][d_c] block is the transposed A), B = q^C_i
-// (K-major, token rows).  Tokens on N = 64.
+// chunk: the head's [d_h][d_c] block is the transposed A) or W^UV_i read
+// K-major (one 128-row x 64-column box per chunk); B = the head's slice of
+// the activations (K-major, token rows).  Tokens on N = 64.
 //
 // Warps (192 threads):
 //   0     TMA producer
 //   1     MMA issuer (one thread) and TMEM owner
 //   2..5  epilogue: TMEM -> bf16 -> shared staging [token][row] -> 16-byte
-//         stores of q_lat rows
+//         stores of the output rows
 // All waits are bounded.
 #pragma once
 
@@ -30,11 +34,13 @@
 namespace mla {
 
 struct HeadsArgs {
-  int n_h, d_h, d_c, T;   // heads, K, latent width (rows of q_lat per head), tokens
-  int k_chunks;           // d_h / 64
-  int m_tiles, n_tiles;   // d_c / 128 row tiles, ceil(T / 64) token tiles
+  int n_h, T;             // heads, tokens
+  int a_rows_per_head;    // rows of A per head: K (MN-major, W^UK: d_h) or M (K-major, W^UV: d_h)
+  int k_chunks;           // K / 64
+  int m_tiles, n_tiles;   // output row tiles per head (of 128), ceil(T / 64) token tiles
   int units;              // n_h * m_tiles * n_tiles
-  __nv_bfloat16* out;     // q_lat [T][n_h][d_c]
+  int out_rows;           // output rows per head (m_tiles * 128)
+  __nv_bfloat16* out;     // [T][n_h][out_rows]
 };
 
 struct HeadsCfg {
@@ -53,9 +59,10 @@ struct HeadsCfg {
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
+template <bool A_MN>
 __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
-    mla_absorb_heads_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
-                            const HeadsArgs a) {
+    mla_heads_gemm_kernel(const __grid_constant__ CUtensorMap mA, const __grid_constant__ CUtensorMap mB,
+                          const HeadsArgs a) {
   using C = HeadsCfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -111,11 +118,15 @@ __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
         int z, m, nt;
         unit(u, &z, &m, &nt);
         for (int kc = 0; kc < a.k_chunks && i < C::NST; ++kc, ++i) {
-          tma_prefetch_l2_2d(&mA, m * 128, z * a.d_h + kc * 64);
-          tma_prefetch_l2_2d(&mA, m * 128 + 64, z * a.d_h + kc * 64);
+          if (A_MN) {
+            tma_prefetch_l2_2d(&mA, m * 128, z * a.a_rows_per_head + kc * 64);
+            tma_prefetch_l2_2d(&mA, m * 128 + 64, z * a.a_rows_per_head + kc * 64);
+          } else {
+            tma_prefetch_l2_3d(&mA, 0, z * a.a_rows_per_head + m * 128, kc);
+          }
         }
       }
-      pdl_wait();  // q^C comes from the kernel before
+      pdl_wait();  // the activations come from the kernel before
       i = 0;
       bool ok = true;
       for (int u = u0; ok && u < u1; ++u) {
@@ -129,8 +140,12 @@ __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
           }
           uint8_t* st = smem + s * C::STAGE;
           mbar_expect_tx(&full[s], C::STAGE);
-          tma_load_2d(st, &mA, &full[s], m * 128, z * a.d_h + kc * 64);
-          tma_load_2d(st + 8192, &mA, &full[s], m * 128 + 64, z * a.d_h + kc * 64);
+          if (A_MN) {
+            tma_load_2d(st, &mA, &full[s], m * 128, z * a.a_rows_per_head + kc * 64);
+            tma_load_2d(st + 8192, &mA, &full[s], m * 128 + 64, z * a.a_rows_per_head + kc * 64);
+          } else {
+            tma_load_3d(st, &mA, &full[s], 0, z * a.a_rows_per_head + m * 128, kc);
+          }
           tma_load_3d(st + C::A_BYTES, &mB, &full[s], 0, nt * C::TN, z * a.k_chunks + kc);
         }
       }
@@ -138,7 +153,7 @@ __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t idesc = idesc_bf16_f32(128, C::TN, true, false);
+      const uint32_t idesc = idesc_bf16_f32(128, C::TN, A_MN, false);
       int i = 0;
       bool ok = true;
       for (int u = u0, ul = 0; ok && u < u1; ++u, ++ul) {
@@ -156,7 +171,8 @@ __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = smem_desc(sa + kk * 2048, 8192, 1024, SW128);
+            const uint64_t ad = A_MN ? smem_desc(sa + kk * 2048, 8192, 1024, SW128)
+                                     : smem_desc(sa + kk * 32, 16, 1024, SW128);
             const uint64_t bd = smem_desc(sb + kk * 32, 16, 1024, SW128);
             mma_bf16_ss(tmem + b * C::TN, ad, bd, idesc, (kc | kk) != 0);
           }
@@ -167,7 +183,7 @@ __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    pdl_wait();  // q_lat may be read by the kernel before until it has finished
+    pdl_wait();  // the output may be read by the kernel before until it has finished
     const int q = warp & 3;
     const int row = q * 32 + (threadIdx.x & 31);  // latent row within the tile (TMEM lane)
     const int et = threadIdx.x - 64;                // 0..127
@@ -196,12 +212,12 @@ __global__ void __launch_bounds__(HeadsCfg::THREADS, 1)
 #pragma unroll
       for (int t = 0; t < C::TN; ++t) stage_out[t * 128 + row] = __float2bfloat16_rn(v[t]);
       if (!group_sync(705)) break;
-      // q_lat[t][z][128 m .. 128 m + 127]: 256 contiguous bytes per token
+      // out[t][z][128 m .. 128 m + 127]: 256 contiguous bytes per token
       for (int idx = et; idx < C::TN * 16; idx += 128) {
         const int t = idx >> 4, part = idx & 15;
         const int tok = nt * C::TN + t;
         if (tok < a.T)
-          *reinterpret_cast<uint4*>(a.out + ((long long)tok * a.n_h + z) * a.d_c + m * 128 + part * 8) =
+          *reinterpret_cast<uint4*>(a.out + ((long long)tok * a.n_h + z) * a.out_rows + m * 128 + part * 8) =
               *reinterpret_cast<const uint4*>(stage_out + t * 128 + part * 8);
       }
       // the staging is read by every thread before the next unit overwrites it

@@ -614,6 +614,36 @@ static mla_status_t tc_compress_append(const mla_layer_desc* D, const mla_weight
   return kv_second_pass(D, w, lat, seq_idx, pos, T, cache, st);
 }
 
+// Per-head projection out[t][i][0 .. 128 m_tiles) on one persistent CTA per
+// SM (tc_gemm_heads.cuh).  A: W^UK read MN-major (A_MN) or W^UV K-major;
+// B: the activations [T][n_h * K].
+template <bool A_MN>
+static mla_status_t run_heads(const void* w, int a_rows, int a_cols, int a_rows_per_head, const void* x, int n_h,
+                              int K, int T, int m_tiles, void* out, cudaStream_t st) {
+  CUtensorMap mA, mB;
+  const bool ok = (A_MN ? map_2d(&mA, w, (uint64_t)a_cols, (uint64_t)a_rows, (uint64_t)a_cols * 2, 64, 64)
+                        : map_rows_chunks(&mA, w, (uint64_t)a_cols, (uint64_t)a_rows, (uint64_t)a_cols * 2, 128, 1)) &&
+                  map_rows_chunks(&mB, x, (uint64_t)n_h * K, (uint64_t)T, (uint64_t)n_h * K * 2,
+                                  (uint32_t)HeadsCfg::TN, 1);
+  if (!ok) return MLA_ERR_CUDA;
+  HeadsArgs ha;
+  ha.n_h = n_h;
+  ha.T = T;
+  ha.a_rows_per_head = a_rows_per_head;
+  ha.k_chunks = K / 64;
+  ha.m_tiles = m_tiles;
+  ha.n_tiles = (T + HeadsCfg::TN - 1) / HeadsCfg::TN;
+  ha.units = n_h * ha.m_tiles * ha.n_tiles;
+  ha.out_rows = m_tiles * 128;
+  ha.out = (__nv_bfloat16*)out;
+  auto kfn = mla_heads_gemm_kernel<A_MN>;
+  cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, HeadsCfg::SMEM);
+  const int grid = std::min(ha.units, num_sms());
+  return launch_pdl(kfn, dim3(grid), dim3(HeadsCfg::THREADS), HeadsCfg::SMEM, st, 1, mA, mB, ha) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
 // [q^C ; q^R] = [W^UQ ; W^QR] c^Q (eq 13 + decoupled query, RoPE on q^R), then
 // (q_lat non-null) q_lat_i = (W^UK_i)^T q^C_i.
 static mla_status_t queries_from_cq(const mla_layer_desc* D, const mla_weights* w, const void* qsrc,
@@ -647,28 +677,10 @@ static mla_status_t queries_from_cq(const mla_layer_desc* D, const mla_weights* 
     if ((s = run_gemm(c, e, plan_q2(D, T), st)) != MLA_OK) return s;
   }
   if (!q_lat) return MLA_OK;  // queries only (the un-absorbed prefill reads q^C)
-  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major, all
-  // (head, row tile, token tile) units on one persistent CTA per SM
-  CUtensorMap mA, mB;
-  if (!map_2d(&mA, w->w_uk, (uint64_t)D->d_c, (uint64_t)D->n_h * D->d_h, (uint64_t)D->d_c * 2, 64, 64) ||
-      !map_rows_chunks(&mB, qc, (uint64_t)nq, (uint64_t)T, (uint64_t)nq * 2, (uint32_t)HeadsCfg::TN, 1))
-    return MLA_ERR_CUDA;
-  HeadsArgs ha;
-  ha.n_h = D->n_h;
-  ha.d_h = D->d_h;
-  ha.d_c = D->d_c;
-  ha.T = T;
-  ha.k_chunks = D->d_h / 64;
-  ha.m_tiles = D->d_c / 128;
-  ha.n_tiles = (T + HeadsCfg::TN - 1) / HeadsCfg::TN;
-  ha.units = D->n_h * ha.m_tiles * ha.n_tiles;
-  ha.out = (__nv_bfloat16*)q_lat;
-  cudaFuncSetAttribute(mla_absorb_heads_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, HeadsCfg::SMEM);
-  const int grid = std::min(ha.units, num_sms());
-  return launch_pdl(mla_absorb_heads_kernel, dim3(grid), dim3(HeadsCfg::THREADS), HeadsCfg::SMEM, st, 1, mA, mB,
-                    ha) == cudaSuccess
-             ? MLA_OK
-             : MLA_ERR_CUDA;
+  // q_lat_i = (W^UK_i)^T q^C_i : per head, A = W^UK_i viewed MN-major (its
+  // [d_h][d_c] block), all (head, row tile, token tile) units on one
+  // persistent CTA per SM; d_c is a multiple of 128 for the bf16 kernels
+  return run_heads<true>(w->w_uk, nq, D->d_c, D->d_h, qc, D->n_h, D->d_h, T, D->d_c / 128, q_lat, st);
 }
 
 // q_c_out: write q^C [T, n_h, d_h] there (the un-absorbed prefill's queries);
@@ -758,7 +770,16 @@ static mla_status_t tc_out_proj(const mla_layer_desc* D, const mla_weights* w, c
   __nv_bfloat16* o = from_o ? (__nv_bfloat16*)o_lat : (__nv_bfloat16*)cv.take((size_t)T * nq * 2);
   if (!from_o && (!ws || !cv.ok())) return MLA_ERR_CAPACITY;
   mla_status_t s;
-  if (!from_o) {  // o_i = W^UV_i o_lat_i  (eq 11 absorbed): per head, A = W^UV_i [d_h, d_c]
+  // With enough heads, o_i = W^UV_i o_lat_i (eq 11 absorbed) runs as one
+  // persistent CTA per SM over the (head, row tile) units, A = W^UV_i
+  // [d_h, d_c] read K-major; few heads (V2-Lite: 16 tiles) keep the batched
+  // GEMM, whose K split over a cluster covers the SMs.
+  const bool per_head = D->d_h % 128 == 0 && D->n_h * (D->d_h / 128) * 2 >= num_sms();
+  if (!from_o && per_head) {
+    if ((s = run_heads<false>(w->w_uv, nq, D->d_c, D->d_h, o_lat, D->n_h, D->d_c, T, D->d_h / 128, o, st)) !=
+        MLA_OK)
+      return s;
+  } else if (!from_o) {  // o_i = W^UV_i o_lat_i as a batched GEMM over the heads
     GemmCall c{};
     c.a0 = w->w_uv;
     c.rows0 = D->d_h;
