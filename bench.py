@@ -307,23 +307,44 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
     code = mla.get_last_error()
     if code != 0:
         raise RuntimeError(f"{name}: device status after warm-up: {mla.status_string(code)}")
+    # whole steps back to back (the throughput), then steps with events around
+    # the attention stage, then (latent form) around the attention kernel alone
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for k in range(steps):
-        one(k)
+        one()
     e1.record(stream)
+    for k in range(steps):
+        one(k)
+    kern = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    if form == "absorbed":
+        for a, b in kern:  # create the events
+            a.record(stream)
+            b.record(stream)
+        for k in range(steps):
+            mla.debug_attention_events(*kern[k])
+            one()
+        mla.debug_attention_events(None, None)
     torch.cuda.synchronize()
     code = mla.get_last_error()
     if code != 0:
         raise RuntimeError(f"{name}: device status after timed steps: {mla.status_string(code)}")
     t_ms = e0.elapsed_time(e1)
     attn_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
-    t_ms, attn_ms = max_over_ranks([t_ms, attn_ms], dev)
+    kern_ms = sum(a.elapsed_time(b) for a, b in kern) / steps if form == "absorbed" else 0.0
+    t_ms, attn_ms, kern_ms = max_over_ranks([t_ms, attn_ms, kern_ms], dev)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     out = {"workload": WORKLOAD_TEXT[name], "value": round(world * rows * steps / (t_ms * 1e-3), 1),
            "unit": "tokens/s", "steps": steps, "warmup": warmup, "ms_per_step": round(t_ms / steps, 4),
            "roofline": roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src)}
     out["roofline"]["traffic"] = committed_traffic(name) if form == "absorbed" else None
+    if form == "absorbed" and kern_ms > 0:
+        k_roof = roofline_of(attn_bytes, attn_flops, kern_ms, peaks, peak_src)
+        kname = ("mla_attn_pair_kernel" if w.dims.n_h == 128 and getattr(w.dims, "cache_dtype", "bf16") != "fp8"
+                 else "mla_attn_kernel")
+        out["roofline"]["kernel_only"] = {"kernel": kname, "us": round(kern_ms * 1e3, 2), "bound": k_roof["bound"],
+                                          "achieved": k_roof["achieved"], "unit": k_roof["unit"],
+                                          "frac": k_roof["frac"]}
     if w.new_tokens > 1:
         out["form"] = form
         if form == "unabsorbed":
