@@ -164,9 +164,11 @@ size_t mla_workspace_size(const mla_layer_desc* desc, int T, int B, int max_kv_l
  *   seq_idx [T] int32     sequence of each token (row of block_table)
  *   pos     [T] int32     position of each token; its page must already be
  *                         in block_table (pos / block_size < max_blocks)
- * Writes cache->pool rows [c^KV (d_c) | RoPE_pos(W^KR h) (d_hr)].
+ * Writes cache->pool rows [c^KV (d_c) | RoPE_pos(W^KR h) (d_hr)] (FP8 rows:
+ * the E4M3 codes of c^KV with the row's scale, see mla_paged_cache).
  * A page id outside [0, num_blocks) sets MLA_ERR_CAPACITY in the device error
- * word and the row is skipped. */
+ * word and the row is skipped.  Workspace: mla_workspace_size(desc, T, 0, 0)
+ * (used with the latent norm or FP8 rows). */
 mla_status_t mla_compress_append(const mla_layer_desc* desc, const mla_weights* w,
                                  const void* h, const int32_t* seq_idx, const int32_t* pos, int T,
                                  mla_paged_cache* cache, void* ws, size_t ws_bytes, void* stream);
@@ -290,7 +292,7 @@ mla_status_t mla_prefill_attn(const mla_layer_desc* desc, const void* q_lat, con
  *   2 n_h d_h bf16 values per pool row), then runs the attention.
  *   q_c, q_rope [B*q_per_seq, n_h, ...] from mla_queries; o [B*q_per_seq, n_h,
  *   d_h] bf16 out; lse [B*q_per_seq, n_h] float out (may be NULL).  bf16 layers
- *   with d_h == 128.
+ *   with d_h == 128 and MLA_CACHE_NATIVE rows.
  * mla_out_proj_unabsorbed: u [T, d] float = W^O o (eq 8) for o [T, n_h, d_h]. */
 size_t mla_prefill_unabsorbed_workspace_size(const mla_layer_desc* desc, int num_blocks, int B, int max_blocks);
 mla_status_t mla_queries(const mla_layer_desc* desc, const mla_weights* w, const void* h, const int32_t* pos, int T,
