@@ -2,7 +2,7 @@
 
     layer = MLALayer(dims, weights)                  # weights: numpy [out, in]
     state = layer.upload(batch)                      # cache pool, page table, h ...
-    u = layer.decode_step(state)                     # a1 -> a2 -> a3 -> a5
+    u = layer.step(state)    # append + queries -> attention (+ LSE combine) -> out_proj
 
 Everything here is buffer management and argument marshalling; the
 arithmetic runs in libmla_b200.so.
