@@ -340,8 +340,7 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
     out["roofline"]["traffic"] = committed_traffic(name) if form == "absorbed" else None
     if form == "absorbed" and kern_ms > 0:
         # the attention kernel alone is the roofline; the stage beside it
-        kname = ("mla_attn_pair_kernel" if w.dims.n_h == 128 and getattr(w.dims, "cache_dtype", "bf16") != "fp8"
-                 else "mla_attn_kernel")
+        kname = "mla_attn_pair_kernel" if w.dims.n_h == 128 else "mla_attn_kernel"
         stage = out["roofline"]
         out["roofline"] = roofline_of(attn_bytes, attn_flops, kern_ms, peaks, peak_src)
         out["roofline"].update({"traffic": stage.pop("traffic"), "kernel": f"{kname} alone (library-recorded events)"})
@@ -559,8 +558,7 @@ def run_ours(args):
 
     if rank == 0:
         traffic = committed_traffic(args.workload)
-        attn_kernel = ("mla_attn_pair_kernel" if w.dims.n_h == 128 and getattr(w.dims, "cache_dtype", "bf16") != "fp8"
-                       else "mla_attn_kernel")
+        attn_kernel = "mla_attn_pair_kernel" if w.dims.n_h == 128 else "mla_attn_kernel"
         # the dominant kernel: the attention kernel alone, between CUDA events
         # the library records on its launch stream around every launch
         roof = roofline_of(attn_bytes, attn_flops, kern_ms, peaks, peak_src)

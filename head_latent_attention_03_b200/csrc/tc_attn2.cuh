@@ -94,16 +94,22 @@ namespace mla {
 #define PAIR_PREFETCH 1  // own pages are prefetched into L2 this many tiles ahead of their load (>= 1)
 #endif
 
-struct PairCfg {
+// F8: the cache rows are FP8 (E4M3 codes of c^KV, bf16 k^R, a power-of-two
+// scale per row); four more warps expand the codes into f16 pair slots.
+template <bool F8>
+struct PairCfgT {
 #if defined(MLA_TRACE) && defined(MLA_TRACE_OBSERVER)
-  static constexpr int THREADS = 256;  // + a barrier-observer warp
+  static constexpr int BASE_THREADS = 256;  // + a barrier-observer warp
 #else
-  static constexpr int THREADS = 224;
+  static constexpr int BASE_THREADS = 224;
 #endif
+  static constexpr int THREADS = BASE_THREADS + (F8 ? 128 : 0);
+  static constexpr int CONV_WARP0 = BASE_THREADS / 32;  // F8: first converter warp
   static constexpr int Q_CHUNK = 64 * 128;        // 64 heads x 64 columns
   static constexpr int Q_BYTES = 9 * Q_CHUNK;     // 72 KB
-  static constexpr int P_BYTES = 2 * 64 * 128;    // staging: 64 heads x 2 pages x 64 tokens (bf16)
+  static constexpr int P_BYTES = 2 * 64 * 128;    // staging: 64 heads x 2 pages x 64 tokens (bf16 or f16)
   static constexpr int PAIR = 16384;              // one page x 2 latent chunks
+  static constexpr int CODES = 8192;              // F8: one page x 128 codes, in the slot's upper half
   static constexpr int ROPE = 8192;               // one page x 64 RoPE columns
   static constexpr int NP = 8;                    // pair slots (two tiles)
   static constexpr int OFF_Q = 0;
@@ -111,7 +117,10 @@ struct PairCfg {
   static constexpr int OFF_ROPE = OFF_P + P_BYTES;
   static constexpr int OFF_PAIR = OFF_ROPE + ROPE;
   static constexpr int OFF_BAR = OFF_PAIR + NP * PAIR;
-  static constexpr int N_BAR = 4 * NP + 1 + 1 + 2 + 2 + 2 + 2 + 2 + 1 + 2;
+  // own_full, oth_full, qk_done, pv_slot [NP]; rope_full, q_full, grp_bar;
+  // s_full, s_free, p_full, pv_done [2]; then either last_ready, z_land [2]
+  // (bf16 rows) or own_land, oth_land [NP] and q_land (F8 rows)
+  static constexpr int N_BAR = 4 * NP + 3 + 4 * 2 + (F8 ? 2 * NP + 1 : 2 * 2);
   static constexpr int OFF_MISC = OFF_BAR + N_BAR * 8;
   static constexpr int OFF_RED = OFF_MISC + 16;
   static constexpr int SMEM = OFF_RED + 3 * 128 * 4 + 1024;
@@ -119,12 +128,17 @@ struct PairCfg {
   static_assert(OFF_P % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_PAIR % 1024 == 0, "1 KB alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
+using PairCfg = PairCfgT<false>;
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
+// m_page1: RoPE chunks of the cached rows (bf16, 128-byte chunks of a row);
+// m_page2: bf16 rows as 4D {column, slot, chunk, block} (2-chunk boxes), or
+// F8 rows as bytes {byte, slot, block} (128-code boxes, no swizzle).
+template <bool F8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREADS, 1)
     mla_attn_pair_kernel(const __grid_constant__ CUtensorMap m_qlat, const __grid_constant__ CUtensorMap m_qrope,
                          const __grid_constant__ CUtensorMap m_page1, const __grid_constant__ CUtensorMap m_page2,
                          const AttnArgs a) {
-  using C = PairCfg;
+  using C = PairCfgT<F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -134,23 +148,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   // next own-page load may overwrite it), s_full (S ready; the RoPE slot is
   // free) and pv_done (O is stable, the tile's P buffer is free).  s_full and
   // pv_done have one instance per tile parity so that a waiter is never two
-  // phases behind.
-  uint64_t* own_full = bar;                   // leader [NP]: own-page pair landed in the slot
-  uint64_t* oth_full = own_full + C::NP;      // leader [NP]: other-page refill landed
+  // phases behind.  With F8 rows own_full, oth_full and q_full count the
+  // converter warps that finished the slot (the codes land on each CTA's own
+  // own_land / oth_land / q_land).
+  uint64_t* own_full = bar;                   // leader [NP]: own-page pair ready in the slot
+  uint64_t* oth_full = own_full + C::NP;      // leader [NP]: other-page refill ready
   uint64_t* qk_done = oth_full + C::NP;       // both [NP]: pair commit once QK has read the slot
-  uint64_t* rope_full = qk_done + C::NP;      // leader
+  uint64_t* pv_slot = qk_done + C::NP;        // both [NP]: pair commit once PV has read the slot
+  uint64_t* rope_full = pv_slot + C::NP;      // leader
   uint64_t* q_full = rope_full + 1;           // leader
-  uint64_t* s_full = q_full + 1;              // both [2]: pair commit after QK(j)
+  uint64_t* grp_bar = q_full + 1;             // local: 128 softmax threads
+  uint64_t* s_full = grp_bar + 1;             // both [2]: pair commit after QK(j)
   uint64_t* s_free = s_full + 2;              // leader [2]: one arrive per CTA
   uint64_t* p_full = s_free + 2;              // leader [2]: P(j) in TMEM, one arrive per softmax warp
   uint64_t* pv_done = p_full + 2;             // both [2]: pair commit after PV(j)
-  uint64_t* last_ready = pv_done + 2;         // leader [2]: both CTAs zeroed the last tile
-  uint64_t* grp_bar = last_ready + 2;         // local: 128 softmax threads
-  uint64_t* z_land = grp_bar + 1;             // local [2]: last tile's other-page refills
-  uint64_t* pv_slot = z_land + 2;             // both [NP]: pair commit once PV has read the slot
+  uint64_t* last_ready = pv_done + 2;         // bf16 rows, leader [2]: both CTAs zeroed the last tile
+  uint64_t* z_land = last_ready + 2;          // bf16 rows, local [2]: last tile's other-page refills
+  uint64_t* own_land = pv_done + 2;           // F8 rows, local [NP]: own-page codes landed
+  uint64_t* oth_land = own_land + C::NP;      // F8 rows, local [NP]: other-page codes landed
+  uint64_t* q_land = oth_land + C::NP;        // F8 rows, local: the segment's queries landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);  // [3][128]: tile max x2, final sums
+  (void)last_ready;
+  (void)z_land;
+  (void)own_land;
+  (void)oth_land;
+  (void)q_land;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -161,23 +185,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   (void)tunit;
 
   if (threadIdx.x == 0) {
+    // F8: a slot or the queries are ready once both CTAs' converter warps of
+    // that kind arrived (two own-page warps per CTA; two refill warps of the
+    // one CTA that refills the slot)
     for (int i = 0; i < C::NP; ++i) {
-      mbar_init(&own_full[i], 1);
-      mbar_init(&oth_full[i], 1);
+      mbar_init(&own_full[i], F8 ? 4 : 1);
+      mbar_init(&oth_full[i], F8 ? 2 : 1);
       mbar_init(&qk_done[i], 1);
       mbar_init(&pv_slot[i], 1);
     }
     mbar_init(rope_full, 1);
-    mbar_init(q_full, 1);
+    mbar_init(q_full, F8 ? 4 : 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 2);
       mbar_init(&pv_done[i], 1);
-      mbar_init(&z_land[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(&p_full[i], PAIR_WARP_ARRIVE ? 8 : 2);
-      mbar_init(&last_ready[i], 2);
+    }
+    if (F8) {
+      for (int i = 0; i < C::NP; ++i) {
+        mbar_init(&own_land[i], 1);
+        mbar_init(&oth_land[i], 1);
+      }
+      mbar_init(q_land, 1);
+    } else {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&z_land[i], 1);
+        mbar_init(&last_ready[i], 2);
+      }
     }
     mbar_init(grp_bar, 128);
     *abort_flag = 0;
@@ -196,7 +231,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   if (threadIdx.x == 0) MLA_TRACE_EVENT(tunit, 0, 0);
   const uint32_t tS = tmem;         // S buffers: columns [0,64) and [64,128)
   const uint32_t tO = tmem + 128;   // O: columns [128,256) (d_c 0..255) and [256,384) (256..511)
-  const uint32_t tP = tmem + 384;   // P buffers (bf16, A operand of PV): columns [384,448) and [448,512)
+  const uint32_t tP = tmem + 384;   // P buffers (bf16 / F8: f16, A operand of PV): columns [384,448) and [448,512)
 
   // cache block of page `page` of the cursor's row; past the row: num_blocks
   // (out of range: TMA reads zeros)
@@ -268,7 +303,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       // Own pages are prefetched into L2 PAIR_PREFETCH tiles ahead (one tile
       // measured best): the loads below, and the other CTA's refills from
       // this page, then see L2 rather than HBM latency.
-      constexpr uint32_t PAGE_BYTES = 64u * (ATT_DC + ATT_DR) * 2u;
+      constexpr uint32_t PAGE_BYTES = 64u * (F8 ? fp8_row_bytes(ATT_DC, ATT_DR) : (ATT_DC + ATT_DR) * 2u);
+      constexpr int ROPE_CHUNK = (F8 ? ATT_DC : 2 * ATT_DC) / 128;  // the 128-byte chunk of a row holding k^R
       TileCursor c, cf;
       c.init(a, range);
       cf = c;
@@ -297,9 +333,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             ok = false;
             break;
           }
-          if (rank == 0) mbar_expect_tx(&own_full[s], 2 * C::PAIR);
-          tma_load_4d_pair(smem + C::OFF_PAIR + s * C::PAIR, &m_page2, mapa_shared(smem_u32(&own_full[s]), 0), 0, 0,
-                           2 * k, blk);
+          if (F8) {
+            // the codes of latent columns 128k .. 128k+127 into the slot's upper half
+            mbar_expect_tx(&own_land[s], C::CODES);
+            tma_load_3d(smem + C::OFF_PAIR + s * C::PAIR + C::CODES, &m_page2, &own_land[s], 128 * k, 0, blk);
+          } else {
+            if (rank == 0) mbar_expect_tx(&own_full[s], 2 * C::PAIR);
+            tma_load_4d_pair(smem + C::OFF_PAIR + s * C::PAIR, &m_page2, mapa_shared(smem_u32(&own_full[s]), 0), 0,
+                             0, 2 * k, blk);
+          }
           if (k == 0) MLA_TRACE_EVENT(tunit, 1, g);
           if (k == 3) MLA_TRACE_EVENT(tunit, 2, g);
         }
@@ -308,14 +350,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
         // QK(g-1) is done (QK reads the RoPE chunk last)
         if (g >= 1 && !mbar_wait(&s_full[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag, 503)) break;
         if (c.first()) {
-          if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
           const int qrow = c.S.r * a.n_h + head0;
-          for (int k = 0; k < 8; ++k)
-            tma_load_2d_pair(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, lq, k * 64, qrow);
-          tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
+          if (F8) {
+            // each CTA's own queries, turned into f16 by its converters
+            mbar_expect_tx(q_land, C::Q_BYTES);
+            for (int k = 0; k < 8; ++k) tma_load_2d(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, q_land, k * 64, qrow);
+            tma_load_2d(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, q_land, 0, qrow);
+          } else {
+            if (rank == 0) mbar_expect_tx(q_full, 2 * C::Q_BYTES);
+            for (int k = 0; k < 8; ++k)
+              tma_load_2d_pair(smem + C::OFF_Q + k * C::Q_CHUNK, &m_qlat, lq, k * 64, qrow);
+            tma_load_2d_pair(smem + C::OFF_Q + 8 * C::Q_CHUNK, &m_qrope, lq, 0, qrow);
+          }
         }
         if (rank == 0) mbar_expect_tx(rope_full, 2 * C::ROPE);
-        tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, 8, blk);
+        tma_load_4d_pair(smem + C::OFF_ROPE, &m_page1, l_rope, 0, 0, ROPE_CHUNK, blk);
         MLA_TRACE_EVENT(tunit, 19, g);
         c.step(a);
       }
@@ -330,7 +379,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
     bool ok = true;
     while (ok && !c.done()) {
       const int g = c.g;
-      const bool zero = c.zero();
+      // F8: the converters zero the rows past kv_len of every slot they write
+      const bool zero = !F8 && c.zero();
       if (lane == 0) {
         int zk = 0;  // refills of this tile that land on z_land
         for (int k = 0; k < 4 && ok; ++k) {
@@ -342,7 +392,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           const int b = page_block(c, c.tok() / 64 + (k & 1));
           const int c0 = 2 * (2 * (k >> 1) + (int)rank);  // columns this CTA multiplies in instruction k >> 1
           uint8_t* dst = smem + C::OFF_PAIR + s * C::PAIR;
-          if (!zero) {
+          if (F8) {
+            // the codes of those columns into the slot's upper half, for this CTA's converters
+            mbar_expect_tx(&oth_land[s], C::CODES);
+            tma_load_3d(dst + C::CODES, &m_page2, &oth_land[s], 64 * c0, 0, b);
+          } else if (!zero) {
             if (rank == 0) mbar_expect_tx(&oth_full[s], C::PAIR);  // the peer's are posted by the MMA issuer
             tma_load_4d_pair(dst, &m_page2, mapa_shared(smem_u32(&oth_full[s]), 0), 0, 0, c0, b);
           } else {
@@ -386,8 +440,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (rank == 0 && elect_one()) {
-      const uint32_t id_qk = idesc_bf16_f32(128, 128, false, false);
-      const uint32_t id_pv = idesc_bf16_f32(128, 256, false, true);
+      // F8: the latent chunks of Q and K, P and V are f16; the RoPE chunk stays bf16
+      const uint32_t id_qr = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t id_qk = F8 ? idesc_f16_f32(128, 128, false, false) : id_qr;
+      const uint32_t id_pv = F8 ? idesc_f16_f32(128, 256, false, true) : idesc_bf16_f32(128, 256, false, true);
       const uint32_t q_base = smem_u32(smem + C::OFF_Q);
       const uint32_t rope_base = smem_u32(smem + C::OFF_ROPE);
       const uint32_t pair0 = smem_u32(smem + C::OFF_PAIR);
@@ -399,7 +455,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
       // posted here, each as soon as the slot's previous refill has been
       // consumed by PV; the leader's own refills post theirs themselves.
       auto post_peer_refill = [&](int k) {
-        if (!cpost.done() && !cpost.zero()) mbar_expect_tx(&oth_full[slot_of(cpost.g, k)], C::PAIR);
+        if (!F8 && !cpost.done() && !cpost.zero()) mbar_expect_tx(&oth_full[slot_of(cpost.g, k)], C::PAIR);
       };
       for (int t = 0; t < 2; ++t) {
         post_peer_refill(0);
@@ -425,7 +481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             if (p_ok) MLA_TRACE_EVENT(tunit, 15, jp);
           }
           if (p_ok) {
-            const bool zero = cp.zero();
+            const bool zero = !F8 && cp.zero();
             while (pv_k < 4) {
               const int s = slot_of(jp, pv_k), u = use_of(jp, pv_k);
               const bool ready = zero ? PAIR_TEST(smem_u32(&last_ready[nz & 1]), (nz >> 1) & 1)
@@ -501,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = smem_desc(q_base + 8 * C::Q_CHUNK + kk * 32, 16, 1024, SW128);
               const uint64_t bd = smem_desc(rope_base + kk * 32, 16, 1024, SW128);
-              mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qk, 1u);
+              mma_bf16_pair(tS + (jq & 1) * 64, ad, bd, id_qr, 1u);
             }
             MLA_TRACE_EVENT(tunit, 7, jq);
             mma_commit_pair(&s_full[jq & 1]);
@@ -528,6 +584,111 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           }
         }
       }
+    }
+  } else if (F8 && warp >= C::CONV_WARP0) {
+    // ------------------------------------------------------------ F8 converters
+    // Two groups of two warps, thread = token row r of a page.  The own group
+    // expands the four own-page pairs of every tile (and, per segment, turns
+    // the queries' latent chunks into f16 in place); the refill group expands
+    // the two pairs this CTA refills from the other page.  A thread reads its
+    // row's 128 codes from the slot's upper half and writes code * 2^e as f16
+    // into both halves in the MMA's SW128 layout: columns 0..63 to the lower
+    // half, 64..127 over exactly the bytes it has just read.  Rows past kv_len
+    // are written as zeros (PV multiplies them by P = 0, and a stale code may
+    // be a NaN).  The values are exact for row scales 2^e, -15 <= e <= 7.
+    const int ct = threadIdx.x - 32 * C::CONV_WARP0;
+    const int grp = ct >> 6, r = ct & 63;
+    constexpr int ROWB = fp8_row_bytes(ATT_DC, ATT_DR);
+    auto row_scale = [&](int blk, int nvalid) -> float {
+      if (r >= nvalid || blk >= a.num_blocks) return 0.f;
+      return *reinterpret_cast<const float*>(a.pool + ((size_t)blk * 64 + r) * ROWB + fp8_scale_off(ATT_DC, ATT_DR));
+    };
+    auto expand = [&](int s, uint32_t sc2, bool valid) {
+      uint8_t* row = smem + C::OFF_PAIR + s * C::PAIR + r * 128;
+      const uint4* in = reinterpret_cast<const uint4*>(row + C::CODES);
+      // thread r takes its row's 16-byte units in the order r, r+1, ... (mod
+      // 8), so the rows of a warp spread over all banks
+      uint4 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = in[(j + r) & 7];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // codes 16k .. 16k+15: f16 columns 16(k%4) .. +15 of half k/4, 16-byte units 2(k%4), 2(k%4)+1
+        const int k = (j + r) & 7;
+        uint8_t* half = row + (k >> 2) * C::CODES;
+        const uint32_t u0 = 2u * (k & 3);
+        uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+        if (valid) {
+          lo = make_uint4(f16x2_from_e4m3x2((uint16_t)v[j].x, sc2), f16x2_from_e4m3x2((uint16_t)(v[j].x >> 16), sc2),
+                          f16x2_from_e4m3x2((uint16_t)v[j].y, sc2), f16x2_from_e4m3x2((uint16_t)(v[j].y >> 16), sc2));
+          hi = make_uint4(f16x2_from_e4m3x2((uint16_t)v[j].z, sc2), f16x2_from_e4m3x2((uint16_t)(v[j].z >> 16), sc2),
+                          f16x2_from_e4m3x2((uint16_t)v[j].w, sc2), f16x2_from_e4m3x2((uint16_t)(v[j].w >> 16), sc2));
+        }
+        *reinterpret_cast<uint4*>(half + ((u0 ^ (uint32_t)(r & 7)) << 4)) = lo;
+        *reinterpret_cast<uint4*>(half + (((u0 + 1) ^ (uint32_t)(r & 7)) << 4)) = hi;
+      }
+    };
+    // one arrive per warp on the leader's barrier, after every lane's writes
+    // are visible to the tensor core
+    auto announce = [&](uint64_t* b) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(b);
+        else
+          PAIR_ARRIVE(mapa_shared(smem_u32(b), 0));
+      }
+    };
+    TileCursor c;
+    c.init(a, range);
+    bool ok = true;
+    while (ok && !c.done()) {
+      const int g = c.g;
+      if (grp == 0) {
+        if (c.first()) {
+          // every lane leaves a wait before its warp's __syncwarp: give up as a warp
+          if (!__all_sync(0xffffffffu, mbar_wait(q_land, c.n & 1, abort_flag, 531))) break;
+          uint4* qv = reinterpret_cast<uint4*>(smem + C::OFF_Q);
+          for (int i = r; i < 8 * C::Q_CHUNK / 16; i += 64) {
+            const uint4 w = qv[i];
+            qv[i] = make_uint4(f16x2_from_bf16x2(w.x), f16x2_from_bf16x2(w.y), f16x2_from_bf16x2(w.z),
+                               f16x2_from_bf16x2(w.w));
+          }
+          announce(q_full);
+        }
+        const int page = c.tok() / 64 + (int)rank;
+        const int blk = page_block(c, page);
+        const int nvalid = min(64, max(0, c.S.kv - 64 * page));
+        const float sc = row_scale(blk, nvalid);
+        const uint32_t sc2 = pack_f16(sc, sc);
+        for (int k = 0; k < 4; ++k) {
+          const int s = slot_of(g, k);
+          if (!__all_sync(0xffffffffu, mbar_wait(&own_land[s], use_of(g, k) & 1, abort_flag, 532))) {
+            ok = false;
+            break;
+          }
+          expand(s, sc2, r < nvalid);
+          announce(&own_full[s]);
+        }
+      } else {
+        // this CTA refills pairs k with (k & 1) != rank: the other page's tokens
+        const int page = c.tok() / 64 + (int)(rank ^ 1u);
+        const int blk = page_block(c, page);
+        const int nvalid = min(64, max(0, c.S.kv - 64 * page));
+        const float sc = row_scale(blk, nvalid);
+        const uint32_t sc2 = pack_f16(sc, sc);
+        for (int k = (int)(rank ^ 1u); k < 4; k += 2) {
+          const int s = slot_of(g, k);
+          if (!__all_sync(0xffffffffu, mbar_wait(&oth_land[s], use_of(g, k) & 1, abort_flag, 533))) {
+            ok = false;
+            break;
+          }
+          expand(s, sc2, r < nvalid);
+          announce(&oth_full[s]);
+        }
+      }
+      c.step(a);
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -614,7 +775,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg::THREADS, 1)
           const float p0 = exp2_approx(s[8 * cc + 2 * e] - m_run);
           const float p1 = exp2_approx(s[8 * cc + 2 * e + 1] - m_run);
           l_run += p0 + p1;
-          pk[cc][e] = pack_bf16(p0, p1);
+          pk[cc][e] = F8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
         }
       }
       // Both TMEM lanes of a head (h and 64 + h) must hold P over all 128

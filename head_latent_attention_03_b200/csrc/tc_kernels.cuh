@@ -101,6 +101,21 @@ inline bool map_cache_chunks(CUtensorMap* m, const void* pool, int num_blocks, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// FP8 cache rows (row_bytes each) as bf16 elements in 128-byte chunks
+// {column in chunk, slot, chunk, block}: chunk d_c / 128 is k^R (64 x 64
+// boxes, 128-byte swizzle), the layout of map_cache_chunks' RoPE box.
+inline bool map_fp8_rope_chunks(CUtensorMap* m, const void* pool, int num_blocks, int row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {64, 64, (cuuint64_t)(row_bytes / 128), (cuuint64_t)num_blocks};
+  cuuint64_t strides[3] = {(cuuint64_t)row_bytes, 128, (cuuint64_t)row_bytes * 64};
+  cuuint32_t box[4] = {64, 64, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(pool), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // FP8 cache rows (row_bytes each) as bytes {byte, slot, block}; box = box_bytes
 // x 64 slots of one page, no swizzle (the codes of 128 latent columns, or a
 // row's 16-byte scale field).
@@ -399,11 +414,14 @@ inline size_t ws_out(const mla_layer_desc* D, int T) {
 }
 
 inline int heads_per_cta(const mla_layer_desc* D) { return D->n_h == 16 ? 16 : 32; }
-// 128-head layers with bf16 rows run on CTA pairs (tc_attn2.cuh), one pair
-// per (row, split); over FP8 rows they run on the one-CTA kernel as four
-// 32-head groups per worker, side by side on the same tiles (L2 serves the
-// other three groups).
-inline bool use_pair_kernel(const mla_layer_desc* D) { return D->n_h == 128 && !fp8_cache(D); }
+// 128-head layers run on CTA pairs (tc_attn2.cuh), one pair per (row,
+// split), over bf16 or FP8 rows.  MLA_FP8_PAIR=0 sends 128-head layers over
+// FP8 rows to the one-CTA kernel instead, as four 32-head groups per worker
+// side by side on the same tiles (L2 serves the other three groups).
+#ifndef MLA_FP8_PAIR
+#define MLA_FP8_PAIR 1
+#endif
+inline bool use_pair_kernel(const mla_layer_desc* D) { return D->n_h == 128 && (MLA_FP8_PAIR || !fp8_cache(D)); }
 
 // Host side of the attention work plan (the device side is
 // mla_attn_plan_kernel).  Automatic decode plans deal the tiles of all rows
@@ -1021,14 +1039,24 @@ static mla_status_t tc_attention(const mla_layer_desc* D, const void* q_lat, con
   cudaError_t e;
   if (g_attn_ev_before && cudaEventRecord(g_attn_ev_before, st) != cudaSuccess) return MLA_ERR_CUDA;
   if (pair) {
-    CUtensorMap m1, m2;
-    if (!map_cache_chunks(&m1, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 1) ||
-        !map_cache_chunks(&m2, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 2))
-      return MLA_ERR_CUDA;
     dim3 grid(2 * p.workers);
-    cudaFuncSetAttribute(mla_attn_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
     // cluster dimensions are compiled in (__cluster_dims__)
-    e = launch_pdl(mla_attn_pair_kernel, grid, dim3(PairCfg::THREADS), PairCfg::SMEM, st, 1, mq, mr, m1, m2, a);
+    if (f8) {
+      // RoPE chunks through a bf16 view of the rows; the codes as bytes (mc)
+      CUtensorMap m1;
+      if (!map_fp8_rope_chunks(&m1, cache->pool, cache->num_blocks, cache_row_bytes(D))) return MLA_ERR_CUDA;
+      using PC = PairCfgT<true>;
+      cudaFuncSetAttribute(mla_attn_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::SMEM);
+      e = launch_pdl(mla_attn_pair_kernel<true>, grid, dim3(PC::THREADS), PC::SMEM, st, 1, mq, mr, m1, mc, a);
+    } else {
+      CUtensorMap m1, m2;
+      if (!map_cache_chunks(&m1, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 1) ||
+          !map_cache_chunks(&m2, cache->pool, cache->num_blocks, ATT_DC + ATT_DR, 2))
+        return MLA_ERR_CUDA;
+      cudaFuncSetAttribute(mla_attn_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
+      e = launch_pdl(mla_attn_pair_kernel<false>, grid, dim3(PairCfg::THREADS), PairCfg::SMEM, st, 1, mq, mr, m1, m2,
+                     a);
+    }
   } else {
     dim3 grid(p.workers * attn_groups(D));
     e = H == 16 ? launch_attn<16>(mq, mr, mc, mr8, ms8, f8, a, grid, st)

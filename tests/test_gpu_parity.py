@@ -446,8 +446,24 @@ def test_fp8_decode_with_latent_norm():
 
 
 def test_fp8_decode_v2_small():
-    # 128 heads over FP8 rows: the one-CTA kernel as four 32-head groups
+    # 128 heads over FP8 rows: the CTA-pair kernel with its converter warps
     w = dataclasses.replace(I.WORKLOADS["v2_fp8"], name="v2_fp8_small", batch=3, prior="list:127,128,1000")
+    check_decode(w)
+
+
+@pytest.mark.parametrize("splits", [0, 1, 3])
+def test_fp8_decode_v2_page_edges(splits):
+    # kv_len 1, 64, 65, 192 and 1001 on a permuted page table: a tile whose
+    # second page lies past the row, one whose second page holds one row, a
+    # full page followed by an empty one; automatic, one-per-row and explicit
+    # splits
+    w = dataclasses.replace(I.WORKLOADS["v2_fp8"], name="v2_fp8_edges", batch=5, prior="list:0,63,64,191,1000")
+    check_decode(w, num_splits=splits)
+
+
+def test_fp8_decode_v2_with_latent_norm():
+    w = _with_norm(dataclasses.replace(I.WORKLOADS["v2_fp8"], name="v2_fp8_norm", batch=2, prior="list:300,65"),
+                   "v2_fp8_norm")
     check_decode(w)
 
 

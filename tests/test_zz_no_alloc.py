@@ -37,6 +37,7 @@ CASES = [
     # FP8 cache rows, automatic and explicit splits
     (dataclasses.replace(I.WORKLOADS["lite_fp8"], name="lite_fp8_auto", batch=4, prior="list:300,1500,900,64"), 0),
     (dataclasses.replace(I.WORKLOADS["lite_fp8"], name="lite_fp8_splits2", batch=4, prior="list:300,1500,900,64"), 2),
+    (dataclasses.replace(I.WORKLOADS["v2_fp8"], name="v2_fp8_auto", batch=3, prior="list:127,128,3000"), 0),
 ]
 
 
