@@ -122,10 +122,18 @@ def physical_gpu_index(local: int) -> int:
     return local
 
 
-def kernel_source_hash() -> str:
-    """Hash of every source the attention kernels are built from."""
+def attention_sources(workload: str):
+    """The sources the workload's attention kernel is built from: the CTA-pair
+    kernel (128 heads) also takes tc_attn2.cuh."""
+    from head_latent_attention_03_b200 import inputs as I
+    pair = I.WORKLOADS[workload].dims.n_h == 128
+    return ("common.cuh", "tc_attn.cuh") + (("tc_attn2.cuh",) if pair else ())
+
+
+def kernel_source_hash(workload: str) -> str:
+    """Hash of every source the workload's attention kernel is built from."""
     h = hashlib.sha256()
-    for name in ("common.cuh", "tc_attn.cuh", "tc_attn2.cuh"):
+    for name in attention_sources(workload):
         with open(os.path.join(ROOT, "head_latent_attention_03_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -133,14 +141,14 @@ def kernel_source_hash() -> str:
 
 def committed_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
+    taken on the current source of that kernel; else None."""
     p = os.path.join(ROOT, "profiles", "attn_dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("kernel_source_sha256_16") != kernel_source_hash():
+    if not e or e.get("kernel_source_sha256_16") != kernel_source_hash(workload):
         return None
     return e.get("dram_bytes_per_launch")
 

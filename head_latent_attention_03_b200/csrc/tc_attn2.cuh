@@ -36,13 +36,19 @@
 // {column, slot, chunk, block}: per tile and CTA, one RoPE box and four
 // 2-chunk own-page boxes, plus two 2-chunk refill boxes.
 //
-// Warps (224 threads per CTA):
+// Warps (224 threads per CTA, 480 over FP8 rows):
 //   0    own-page producer (four latent pairs per tile as their slots free
 //        up, then the RoPE chunk once QK of the previous tile is done)
 //   1    MMA issuer (leader CTA only, one thread) and TMEM owner (both CTAs)
 //   2-5  softmax: thread = (head, page half of the tile)
 //   6    other-page producer: refills the pair slots PV needs once QK is done
-//        with them; zeroes rows past kv_len in the last tile
+//        with them; zeroes rows past kv_len in the last tile (bf16 rows)
+//   7-14 FP8 rows only: converters.  The producers then load each pair's
+//        128 codes per token (8 KB per page) into the upper half of its slot
+//        and the converters expand them to f16 over the whole slot, own
+//        pages before QK and refills before PV, zeroing rows past kv_len;
+//        QK's latent chunks and PV run as f16 MMAs on f16 queries and P, the
+//        RoPE chunk as a bf16 MMA into the same accumulator.
 // TMA pair loads complete their bytes on the leader's barriers, for which the
 // leader alone posts the byte count; the other CTA's only arrives on the
 // leader's barriers are "S read" (one per tile), "P written" (one per softmax
@@ -94,8 +100,13 @@ namespace mla {
 #define PAIR_PREFETCH 1  // own pages are prefetched into L2 this many tiles ahead of their load (>= 1)
 #endif
 
+#ifndef PAIR_CONV_WARPS
+#define PAIR_CONV_WARPS 8  // F8: converter warps per CTA (4 or 8)
+#endif
+
 // F8: the cache rows are FP8 (E4M3 codes of c^KV, bf16 k^R, a power-of-two
-// scale per row); four more warps expand the codes into f16 pair slots.
+// scale per row); PAIR_CONV_WARPS more warps expand the codes into f16 pair
+// slots.
 template <bool F8>
 struct PairCfgT {
 #if defined(MLA_TRACE) && defined(MLA_TRACE_OBSERVER)
@@ -103,7 +114,9 @@ struct PairCfgT {
 #else
   static constexpr int BASE_THREADS = 224;
 #endif
-  static constexpr int THREADS = BASE_THREADS + (F8 ? 128 : 0);
+  static constexpr int CONV_WARPS = PAIR_CONV_WARPS;
+  static_assert(CONV_WARPS == 4 || CONV_WARPS == 8, "converter warps");
+  static constexpr int THREADS = BASE_THREADS + (F8 ? 32 * CONV_WARPS : 0);
   static constexpr int CONV_WARP0 = BASE_THREADS / 32;  // F8: first converter warp
   static constexpr int Q_CHUNK = 64 * 128;        // 64 heads x 64 columns
   static constexpr int Q_BYTES = 9 * Q_CHUNK;     // 72 KB
@@ -186,8 +199,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREAD
 
   if (threadIdx.x == 0) {
     // F8: a slot or the queries are ready once both CTAs' converter warps of
-    // that kind arrived (two own-page warps per CTA; two refill warps of the
-    // one CTA that refills the slot)
+    // that kind arrived (a slot is expanded by two warps: per CTA for its own
+    // page, by the one CTA that refills it for the other page)
     for (int i = 0; i < C::NP; ++i) {
       mbar_init(&own_full[i], F8 ? 4 : 1);
       mbar_init(&oth_full[i], F8 ? 2 : 1);
@@ -195,7 +208,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREAD
       mbar_init(&pv_slot[i], 1);
     }
     mbar_init(rope_full, 1);
-    mbar_init(q_full, F8 ? 4 : 1);
+    mbar_init(q_full, F8 ? C::CONV_WARPS : 1);  // F8: the own-page half of the converter warps, both CTAs
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 2);
@@ -587,17 +600,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREAD
     }
   } else if (F8 && warp >= C::CONV_WARP0) {
     // ------------------------------------------------------------ F8 converters
-    // Two groups of two warps, thread = token row r of a page.  The own group
-    // expands the four own-page pairs of every tile (and, per segment, turns
-    // the queries' latent chunks into f16 in place); the refill group expands
-    // the two pairs this CTA refills from the other page.  A thread reads its
-    // row's 128 codes from the slot's upper half and writes code * 2^e as f16
-    // into both halves in the MMA's SW128 layout: columns 0..63 to the lower
-    // half, 64..127 over exactly the bytes it has just read.  Rows past kv_len
-    // are written as zeros (PV multiplies them by P = 0, and a stale code may
-    // be a NaN).  The values are exact for row scales 2^e, -15 <= e <= 7.
+    // Units of two warps, thread = token row r of a page.  The first half of
+    // the units expands the four own-page pairs of every tile (and, per
+    // segment, turns the queries' latent chunks into f16 in place); the
+    // second half expands the two pairs this CTA refills from the other page.
+    // With two units per half, unit i of a half takes every second pair.  A
+    // thread reads its row's 128 codes from the slot's upper half and writes
+    // code * 2^e as f16 into both halves in the MMA's SW128 layout: columns
+    // 0..63 to the lower half, 64..127 over exactly the bytes it has just
+    // read.  Rows past kv_len are written as zeros (PV multiplies them by
+    // P = 0, and a stale code may be a NaN).  The values are exact for row
+    // scales 2^e, -15 <= e <= 7.
+    constexpr int NU = C::CONV_WARPS / 4;  // units per half
     const int ct = threadIdx.x - 32 * C::CONV_WARP0;
-    const int grp = ct >> 6, r = ct & 63;
+    const int unit = ct >> 6, r = ct & 63;
+    const bool own_half = unit < NU;
+    const int sg = unit % NU;
     constexpr int ROWB = fp8_row_bytes(ATT_DC, ATT_DR);
     auto row_scale = [&](int blk, int nvalid) -> float {
       if (r >= nvalid || blk >= a.num_blocks) return 0.f;
@@ -645,12 +663,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREAD
     bool ok = true;
     while (ok && !c.done()) {
       const int g = c.g;
-      if (grp == 0) {
+      if (own_half) {
         if (c.first()) {
           // every lane leaves a wait before its warp's __syncwarp: give up as a warp
           if (!__all_sync(0xffffffffu, mbar_wait(q_land, c.n & 1, abort_flag, 531))) break;
           uint4* qv = reinterpret_cast<uint4*>(smem + C::OFF_Q);
-          for (int i = r; i < 8 * C::Q_CHUNK / 16; i += 64) {
+          for (int i = ct; i < 8 * C::Q_CHUNK / 16; i += 64 * NU) {
             const uint4 w = qv[i];
             qv[i] = make_uint4(f16x2_from_bf16x2(w.x), f16x2_from_bf16x2(w.y), f16x2_from_bf16x2(w.z),
                                f16x2_from_bf16x2(w.w));
@@ -662,7 +680,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREAD
         const int nvalid = min(64, max(0, c.S.kv - 64 * page));
         const float sc = row_scale(blk, nvalid);
         const uint32_t sc2 = pack_f16(sc, sc);
-        for (int k = 0; k < 4; ++k) {
+        for (int k = sg; k < 4; k += NU) {
           const int s = slot_of(g, k);
           if (!__all_sync(0xffffffffu, mbar_wait(&own_land[s], use_of(g, k) & 1, abort_flag, 532))) {
             ok = false;
@@ -678,7 +696,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfgT<F8>::THREAD
         const int nvalid = min(64, max(0, c.S.kv - 64 * page));
         const float sc = row_scale(blk, nvalid);
         const uint32_t sc2 = pack_f16(sc, sc);
-        for (int k = (int)(rank ^ 1u); k < 4; k += 2) {
+        for (int k = (int)(rank ^ 1u) + 2 * sg; k < 4; k += 2 * NU) {
           const int s = slot_of(g, k);
           if (!__all_sync(0xffffffffu, mbar_wait(&oth_land[s], use_of(g, k) & 1, abort_flag, 533))) {
             ok = false;
