@@ -40,8 +40,8 @@ bool desc_valid(const mla_layer_desc* D) {
   return D->dtype == MLA_F32 || D->dtype == MLA_BF16;
 }
 
-// Every latent attention path reads both row formats (FP8 rows of a 128-head
-// layer go to the one-CTA kernel, see use_pair_kernel).
+// Every latent attention path reads both row formats (both attention kernels
+// have an FP8 form).
 bool attn_cache_supported(const mla_layer_desc*) { return true; }
 
 // Shapes the tcgen05 kernels are written for.

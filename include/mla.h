@@ -51,8 +51,8 @@
  *  MLA_CACHE_FP8_E4M3: MLA_BF16 layers; the latent attention
  *    (mla_decode_attn, mla_decode_attn_noalloc, mla_decode_attn_partial,
  *    mla_prefill_attn) reads FP8 rows at every supported n_h (128-head
- *    layers as four 32-head groups per CTA set instead of CTA pairs); the
- *    un-absorbed prefill returns MLA_ERR_UNSUPPORTED.
+ *    layers on CTA pairs, as with native rows); the un-absorbed prefill
+ *    returns MLA_ERR_UNSUPPORTED.
  */
 #ifndef MLA_H
 #define MLA_H
