@@ -4,6 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload v2|v2_fp8|lite|lite_fp8|long|prefill] [--no-cpu-baseline] [--no-extra]
 
+--gpus N must match the ranks torch.distributed.run launched (WORLD_SIZE);
+started without it and N > 1, bench.py launches the N ranks itself.
+
 A step is one pass of the whole hot path over one batch: compress_append ->
 absorb_q -> decode attention (+ LSE combine) -> out_proj, through the C ABI.
 Default workload: the DeepSeek-V2-shaped layer, decode batch 64 with cache
@@ -673,6 +676,18 @@ def main():
     ap.add_argument("--profile-run", action="store_true",
                     help="only the timed device steps (for ncu launch lists): no clock sampling, e2e or CPU leg")
     args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus != world:
+        if "RANK" not in os.environ and args.gpus > 1:
+            # one process per GPU: start the ranks under torch.distributed.run
+            import socket
+            with socket.socket() as s:
+                s.bind(("127.0.0.1", 0))
+                port = s.getsockname()[1]
+            cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+                   "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+            sys.exit(subprocess.call(cmd))
+        sys.exit(f"bench.py: --gpus {args.gpus} but {world} rank(s) were launched")
     if args.impl == "reference":
         run_reference(args)
     else:

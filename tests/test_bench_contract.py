@@ -45,3 +45,14 @@ def test_attention_sources_follow_the_kernel():
         assert bench.attention_sources(w) == ("common.cuh", "tc_attn.cuh")
     assert bench.kernel_source_hash("v2") == bench.kernel_source_hash("v2_fp8")
     assert bench.kernel_source_hash("v2") != bench.kernel_source_hash("lite")
+
+
+def test_gpus_flag_must_match_the_launched_ranks():
+    # under torch.distributed.run the rank count is WORLD_SIZE; a different
+    # --gpus is refused before any work
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "4", "--impl", "reference"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert res.returncode != 0
+    assert "--gpus 4 but 2 rank(s)" in res.stderr
+    assert res.stdout.strip() == ""
