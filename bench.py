@@ -142,6 +142,12 @@ def kernel_source_hash(workload: str) -> str:
     return h.hexdigest()[:16]
 
 
+def attention_tokens_per_s(world: int, rows: int, attn_ms: float):
+    """Decode tokens/s of the attention stage alone (plan + attention + LSE
+    combine, one call per step), whole job: every rank's rows per call time."""
+    return round(world * rows / (attn_ms * 1e-3), 1) if attn_ms > 0 else None
+
+
 def committed_traffic(workload: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
     taken on the current source of that kernel; else None."""
@@ -356,7 +362,8 @@ def measure_extra(name, steps, warmup, dev, peaks, peak_src):
         out["roofline"] = roofline_of(attn_bytes, attn_flops, kern_ms, peaks, peak_src)
         out["roofline"].update({"traffic": stage.pop("traffic"), "kernel": f"{kname} alone (library-recorded events)"})
         out["roofline"]["stage"] = {"us": round(attn_ms * 1e3, 2), "bound": stage["bound"], "achieved": stage["achieved"],
-                                    "unit": stage["unit"], "frac": stage["frac"]}
+                                    "unit": stage["unit"], "frac": stage["frac"],
+                                    "tokens_per_s": attention_tokens_per_s(world, rows, attn_ms)}
     if w.new_tokens > 1:
         out["form"] = form
         if form == "unabsorbed":
@@ -580,7 +587,8 @@ def run_ours(args):
         st_roof = roofline_of(attn_bytes, attn_flops, attn_ms, peaks, peak_src)
         roof["stage"] = {"what": f"mla_attn_plan_kernel + {attn_kernel} + mla_combine_kernel between events around "
                                  f"the attention call", "us": round(attn_ms * 1e3, 2), "bound": st_roof["bound"],
-                         "achieved": st_roof["achieved"], "unit": st_roof["unit"], "frac": st_roof["frac"]}
+                         "achieved": st_roof["achieved"], "unit": st_roof["unit"], "frac": st_roof["frac"],
+                         "tokens_per_s": attention_tokens_per_s(world, rows, attn_ms)}
         value = world * rows * args.steps / (t_ms * 1e-3)
         e2e_value = world * rows * e2e_steps / (t_e2e * 1e-3) if e2e_steps else None
         out = {

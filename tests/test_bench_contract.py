@@ -56,3 +56,11 @@ def test_gpus_flag_must_match_the_launched_ranks():
     assert res.returncode != 0
     assert "--gpus 4 but 2 rank(s)" in res.stderr
     assert res.stdout.strip() == ""
+
+
+def test_attention_tokens_per_s_is_whole_job_rows_over_the_stage_time():
+    sys.path.insert(0, ROOT)
+    import bench
+    # 64 rows per call in 0.140 ms on each of 2 ranks
+    assert bench.attention_tokens_per_s(2, 64, 0.140) == round(2 * 64 / 0.140e-3, 1)
+    assert bench.attention_tokens_per_s(1, 64, 0.0) is None
