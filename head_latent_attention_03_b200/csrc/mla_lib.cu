@@ -24,6 +24,20 @@ constexpr int kVersionMajor = 0, kVersionMinor = 1;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// A bounded wait that runs out: one thread waits on a barrier that nothing
+// arrives on, with the kernels' own wait (mbar_wait), so the give-up path
+// (error word, status) can be exercised without stopping a pipeline that has
+// copies or MMAs in flight.
+constexpr long long kProbeMaxNs = 100000000LL;  // 0.1 s
+__global__ void mla_wait_probe_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, nullptr, 901);
+  }
+}
+
 mla_status_t check_launch() {
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
@@ -397,6 +411,22 @@ int mla_trace_read(void* dst, size_t bytes) {
   return cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros)) == cudaSuccess ? (int)bytes : -1;
 }
 #endif
+
+mla_status_t mla_debug_wait_probe(long long limit_ns, void* stream) {
+  if (limit_ns <= 0 || limit_ns > kProbeMaxNs) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  unsigned long long prev = 0;
+  const unsigned long long lim = (unsigned long long)limit_ns;
+  if (cudaMemcpyFromSymbol(&prev, g_spin_limit_ns, sizeof(prev)) != cudaSuccess) return MLA_ERR_CUDA;
+  // pageable sources: each copy is staged before the call returns
+  if (cudaMemcpyToSymbolAsync(g_spin_limit_ns, &lim, sizeof(lim), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  mla_wait_probe_kernel<<<1, 32, 0, st>>>();
+  const cudaError_t e = cudaGetLastError();
+  // the process-wide limit goes back whatever the launch did
+  const cudaError_t r = cudaMemcpyToSymbolAsync(g_spin_limit_ns, &prev, sizeof(prev), 0, cudaMemcpyHostToDevice, st);
+  return e == cudaSuccess && r == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
 
 void mla_debug_attention_events(void* before, void* after) {
   g_attn_ev_before = reinterpret_cast<cudaEvent_t>(before);

@@ -94,6 +94,7 @@ _SIGS = {
                                                ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "mla_cache_row_bytes": (ctypes.c_size_t, [ctypes.POINTER(LayerDesc)]),
     "mla_debug_attention_events": (None, [ctypes.c_void_p, ctypes.c_void_p]),
+    "mla_debug_wait_probe": (ctypes.c_int, [ctypes.c_longlong, ctypes.c_void_p]),
     "mla_compress_append_absorb_q": (ctypes.c_int, [ctypes.POINTER(LayerDesc), ctypes.POINTER(Weights),
                                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                                     ctypes.POINTER(PagedCache), ctypes.c_void_p, ctypes.c_void_p,
@@ -171,6 +172,13 @@ def debug_attention_events(before=None, after=None):
     (so that they exist)."""
     lib().mla_debug_attention_events(before.cuda_event if before is not None else None,
                                      after.cuda_event if after is not None else None)
+
+
+def debug_wait_probe(limit_ns: int, stream=None) -> int:
+    """Run one bounded wait that nothing completes, under a wait limit of
+    limit_ns; returns the call's status (the timeout is read with
+    get_last_error)."""
+    return lib().mla_debug_wait_probe(int(limit_ns), _stream(stream))
 
 
 def cache_row_bytes(desc: LayerDesc) -> int:

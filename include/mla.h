@@ -324,6 +324,18 @@ mla_status_t mla_get_last_error(void* stream);
  * for benchmarks only. */
 void mla_debug_attention_events(void* before, void* after);
 
+/* Test hook for the bounded waits.  Sets the process-wide wait limit of the
+ * kernels to `limit_ns` (1 .. 100,000,000 ns) on `stream`, runs one kernel
+ * whose single thread waits on a shared-memory barrier that nothing arrives
+ * on (the kernels' own wait routine, so it gives up after the limit and
+ * records MLA_ERR_DEVICE_TIMEOUT in the device error word; no copy or MMA is
+ * in flight), then puts the previous limit back on the same stream.  Returns
+ * MLA_ERR_INVALID_ARG for a limit out of range, MLA_ERR_CUDA if a copy or the
+ * launch failed, else MLA_OK; the timeout itself is read with
+ * mla_get_last_error(stream).  Kernels on other streams that run meanwhile
+ * see the lowered limit: for tests only. */
+mla_status_t mla_debug_wait_probe(long long limit_ns, void* stream);
+
 /* Static string for a status code. */
 const char* mla_status_string(mla_status_t status);
 

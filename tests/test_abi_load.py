@@ -56,6 +56,9 @@ def test_invalid_arguments_are_rejected_without_a_gpu(lib):
     bad = mla.layer_desc(V2)
     bad.d_hr = 63  # odd RoPE width
     assert mla.workspace_size(bad, 1, 1, 64) == 0
+    # the wait probe's limit must lie in 1 ns .. 0.1 s; checked before any CUDA call
+    assert mla.lib().mla_debug_wait_probe(0, None) == 1
+    assert mla.lib().mla_debug_wait_probe(100_000_001, None) == 1
 
 
 def test_fp8_cache_rows_and_limits_without_a_gpu(lib):
